@@ -1,0 +1,302 @@
+"""Pins for the fp64 oracle: every check here compares it with something other
+than itself -- hand-derived golden values, closed forms, invariants, finite
+differences, and PyTorch's own fp64 attention routine on the CPU.
+
+Each test is chosen so that a plausible slip in the oracle (a dropped scale, a
+wrong sign, a transposed operand, a wrong head-group map, a causal off-by-one,
+a mix-up of packed sequence offsets) fails at least one of them.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from long_context_attention_fwd_b200 import inputs as I
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def rnd(shape, seed, mult=1.0):
+    return I.normal(I.stream_key(seed, 99), int(np.prod(shape))).reshape(shape) * mult
+
+
+# ---------------------------------------------------------------- golden values
+@pytest.mark.parametrize("fname", ["hand_s2_d1_causal.json", "hand_s2_d1_full.json"])
+def test_golden_hand_derived(fname):
+    g = json.load(open(os.path.join(GOLDEN, fname)))
+    p = g["problem"]
+    shp = (p["S"], 1, p["D"])
+    q = np.array(p["q"], dtype=np.float64).reshape(shp)
+    k = np.array(p["k"], dtype=np.float64).reshape(shp)
+    v = np.array(p["v"], dtype=np.float64).reshape(shp)
+    do = np.array(p["dO"], dtype=np.float64).reshape(shp)
+    o, lse = oracle.fwd(q, k, v, p["causal"], p["scale"], B=1, S=p["S"])
+    dq, dk, dv = oracle.bwd(q, k, v, do, p["causal"], p["scale"], B=1, S=p["S"])
+    e = g["expected"]
+    np.testing.assert_allclose(o.ravel(), e["o"], rtol=0, atol=1e-13)
+    np.testing.assert_allclose(lse.ravel(), e["lse"], rtol=0, atol=1e-13)
+    np.testing.assert_allclose(dq.ravel(), e["dq"], rtol=0, atol=1e-13)
+    np.testing.assert_allclose(dk.ravel(), e["dk"], rtol=0, atol=1e-13)
+    np.testing.assert_allclose(dv.ravel(), e["dv"], rtol=0, atol=1e-13)
+
+
+# ---------------------------------------------------------------- closed forms
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("gqa", [(2, 2), (4, 2), (6, 1)])
+def test_v_ones_gives_ones(causal, gqa):
+    Hq, Hkv = gqa
+    S, D = 37, 8
+    q = rnd((S, Hq, D), 1)
+    k = rnd((S, Hkv, D), 2)
+    v = np.ones((S, Hkv, D))
+    o, _ = oracle.fwd(q, k, v, causal, 0.7, B=1, S=S)
+    np.testing.assert_allclose(o, 1.0, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_identity_values_expose_softmax_rows(causal):
+    # v_j = e_j (S <= D) turns O_i into the probability row P_i.
+    S, D, H = 9, 12, 2
+    q = rnd((S, H, D), 3)
+    k = rnd((S, H, D), 4)
+    v = np.zeros((S, H, D))
+    for j in range(S):
+        v[j, :, j] = 1.0
+    scale = 0.9
+    o, lse = oracle.fwd(q, k, v, causal, scale, B=1, S=S)
+    P = o[:, :, :S]  # [i, h, j]
+    np.testing.assert_allclose(P.sum(-1), 1.0, rtol=0, atol=1e-12)
+    assert (P >= 0).all()
+    np.testing.assert_array_equal(o[:, :, S:], 0.0)
+    for i in range(S):
+        for h in range(H):
+            n = i + 1 if causal else S
+            if causal:
+                np.testing.assert_array_equal(P[i, h, n:], 0.0)
+            # ratios of probabilities are exponentials of score differences
+            s = scale * (k[:n, h, :] @ q[i, h, :])
+            np.testing.assert_allclose(np.log(P[i, h, :n] / P[i, h, 0]), s - s[0], atol=1e-10)
+            # lse is the log of the normaliser: P_ij = exp(s_ij - lse_i)
+            np.testing.assert_allclose(P[i, h, :n], np.exp(s - lse[0, h, i]), rtol=1e-12)
+
+
+def test_identical_keys_causal_prefix_mean():
+    S, H, D = 40, 3, 8
+    q = rnd((S, H, D), 5)
+    kk = rnd((1, H, D), 6)
+    k = np.repeat(kk, S, axis=0)
+    v = rnd((S, H, D), 7)
+    scale = 0.37
+    o, lse = oracle.fwd(q, k, v, True, scale, B=1, S=S)
+    for i in range(S):
+        np.testing.assert_allclose(o[i], v[: i + 1].mean(0), rtol=0, atol=1e-12)
+        for h in range(H):
+            want = scale * float(q[i, h] @ kk[0, h]) + math.log(i + 1)
+            assert abs(lse[0, h, i] - want) < 1e-12
+    # gradients: a uniform softmax has dQ = 0, and dK sums to zero over keys
+    do = rnd((S, H, D), 8)
+    dq, dk, dv = oracle.bwd(q, k, v, do, True, scale, B=1, S=S)
+    np.testing.assert_allclose(dq, 0.0, atol=1e-12)
+    np.testing.assert_allclose(dk.sum(0), 0.0, atol=1e-11)
+    # dV_j = sum_{i>=j} dO_i / (i+1)
+    for j in range(S):
+        want = sum(do[i] / (i + 1) for i in range(j, S))
+        np.testing.assert_allclose(dv[j], want, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_scale_zero_is_mean(causal):
+    S, H, D = 23, 2, 4
+    q = rnd((S, H, D), 9)
+    k = rnd((S, H, D), 10)
+    v = rnd((S, H, D), 11)
+    o, lse = oracle.fwd(q, k, v, causal, 0.0, B=1, S=S)
+    for i in range(S):
+        n = i + 1 if causal else S
+        np.testing.assert_allclose(o[i], v[:n].mean(0), atol=1e-12)
+        np.testing.assert_allclose(lse[0, :, i], math.log(n), atol=1e-12)
+
+
+def test_single_token():
+    Hq, Hkv, D = 4, 2, 8
+    q = rnd((1, Hq, D), 12)
+    k = rnd((1, Hkv, D), 13)
+    v = rnd((1, Hkv, D), 14)
+    do = rnd((1, Hq, D), 15)
+    scale = 0.5
+    o, lse = oracle.fwd(q, k, v, True, scale, B=1, S=1)
+    dq, dk, dv = oracle.bwd(q, k, v, do, True, scale, B=1, S=1)
+    for h in range(Hq):
+        g = h // (Hq // Hkv)
+        np.testing.assert_allclose(o[0, h], v[0, g], atol=1e-14)
+        assert abs(lse[0, h, 0] - scale * float(q[0, h] @ k[0, g])) < 1e-13
+    np.testing.assert_allclose(dq, 0.0, atol=1e-14)
+    np.testing.assert_allclose(dk, 0.0, atol=1e-14)
+    for g in range(Hkv):
+        np.testing.assert_allclose(dv[0, g], do[0, 2 * g] + do[0, 2 * g + 1], atol=1e-14)
+
+
+# ---------------------------------------------------------------- structure
+@pytest.mark.parametrize("causal", [True, False])
+def test_gqa_equals_mha_with_repeated_kv(causal):
+    S, Hq, Hkv, D = 19, 6, 2, 8
+    G = Hq // Hkv
+    q, k, v, do = rnd((S, Hq, D), 16), rnd((S, Hkv, D), 17), rnd((S, Hkv, D), 18), rnd((S, Hq, D), 19)
+    kr, vr = np.repeat(k, G, axis=1), np.repeat(v, G, axis=1)  # head h reads kv head h // G
+    o1, l1 = oracle.fwd(q, k, v, causal, 0.3, B=1, S=S)
+    o2, l2 = oracle.fwd(q, kr, vr, causal, 0.3, B=1, S=S)
+    np.testing.assert_allclose(o1, o2, atol=1e-13)
+    np.testing.assert_allclose(l1, l2, atol=1e-13)
+    dq1, dk1, dv1 = oracle.bwd(q, k, v, do, causal, 0.3, B=1, S=S)
+    dq2, dk2, dv2 = oracle.bwd(q, kr, vr, do, causal, 0.3, B=1, S=S)
+    np.testing.assert_allclose(dq1, dq2, atol=1e-12)
+    np.testing.assert_allclose(dk1, dk2.reshape(S, Hkv, G, D).sum(2), atol=1e-12)
+    np.testing.assert_allclose(dv1, dv2.reshape(S, Hkv, G, D).sum(2), atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_packed_equals_separate(causal):
+    lens = [5, 0, 13, 1, 9]
+    Hq, Hkv, D = 4, 2, 8
+    T = sum(lens)
+    q, k, v, do = rnd((T, Hq, D), 20), rnd((T, Hkv, D), 21), rnd((T, Hkv, D), 22), rnd((T, Hq, D), 23)
+    cu = I.cu_seqlens_from(lens)
+    o, lse = oracle.fwd(q, k, v, causal, 0.4, cu_seqlens=cu)
+    dq, dk, dv = oracle.bwd(q, k, v, do, causal, 0.4, cu_seqlens=cu)
+    for s, L in enumerate(lens):
+        a, b = cu[s], cu[s + 1]
+        if L == 0:
+            continue
+        o1, l1 = oracle.fwd(q[a:b], k[a:b], v[a:b], causal, 0.4, B=1, S=L)
+        g1 = oracle.bwd(q[a:b], k[a:b], v[a:b], do[a:b], causal, 0.4, B=1, S=L)
+        assert np.array_equal(o[a:b], o1)
+        assert np.array_equal(lse[:, a:b], l1[0])
+        assert np.array_equal(dq[a:b], g1[0])
+        assert np.array_equal(dk[a:b], g1[1])
+        assert np.array_equal(dv[a:b], g1[2])
+
+
+def test_batch_equals_separate():
+    B, S, H, D = 3, 11, 2, 4
+    q, k, v = rnd((B * S, H, D), 24), rnd((B * S, H, D), 25), rnd((B * S, H, D), 26)
+    o, lse = oracle.fwd(q, k, v, True, 0.5, B=B, S=S)
+    for b in range(B):
+        sl = slice(b * S, (b + 1) * S)
+        o1, l1 = oracle.fwd(q[sl], k[sl], v[sl], True, 0.5, B=1, S=S)
+        assert np.array_equal(o[sl], o1)
+        assert np.array_equal(lse[b], l1[0])
+
+
+def test_noncausal_key_permutation_invariance():
+    S, H, D = 17, 2, 8
+    q, k, v = rnd((S, H, D), 27), rnd((S, H, D), 28), rnd((S, H, D), 29)
+    perm = np.random.default_rng(0).permutation(S)
+    o1, l1 = oracle.fwd(q, k, v, False, 0.6, B=1, S=S)
+    o2, l2 = oracle.fwd(q, k[perm], v[perm], False, 0.6, B=1, S=S)
+    np.testing.assert_allclose(o1, o2, atol=1e-13)
+    np.testing.assert_allclose(l1, l2, atol=1e-13)
+
+
+def test_causal_row_ignores_future_keys():
+    # Changing keys/values after position i leaves rows <= i untouched.
+    S, H, D = 16, 2, 4
+    q, k, v = rnd((S, H, D), 30), rnd((S, H, D), 31), rnd((S, H, D), 32)
+    o1, l1 = oracle.fwd(q, k, v, True, 0.5, B=1, S=S)
+    k2, v2 = k.copy(), v.copy()
+    k2[9:] += 3.0
+    v2[9:] -= 2.0
+    o2, l2 = oracle.fwd(q, k2, v2, True, 0.5, B=1, S=S)
+    assert np.array_equal(o1[:9], o2[:9])
+    assert not np.allclose(o1[9:], o2[9:])
+
+
+# ---------------------------------------------------------------- gradients
+@pytest.mark.parametrize("causal", [True, False])
+def test_finite_differences(causal):
+    S, Hq, Hkv, D = 7, 4, 2, 3
+    scale = 0.8
+    q, k, v, do = rnd((S, Hq, D), 33), rnd((S, Hkv, D), 34), rnd((S, Hkv, D), 35), rnd((S, Hq, D), 36)
+
+    def loss(q_, k_, v_):
+        o, _ = oracle.fwd(q_, k_, v_, causal, scale, B=1, S=S)
+        return float((o * do).sum())
+
+    dq, dk, dv = oracle.bwd(q, k, v, do, causal, scale, B=1, S=S)
+    h = 1e-6
+    for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        fd = np.zeros_like(x)
+        for idx in np.ndindex(*x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            args_p = {"q": q, "k": k, "v": v}
+            args_m = dict(args_p)
+            args_p[name], args_m[name] = xp, xm
+            fd[idx] = (loss(args_p["q"], args_p["k"], args_p["v"])
+                       - loss(args_m["q"], args_m["k"], args_m["v"])) / (2 * h)
+        rel = np.linalg.norm(fd - g) / np.linalg.norm(g)
+        assert rel < 1e-6, (name, rel)
+
+
+# ---------------------------------------------------------------- library routine
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("gqa", [(4, 4), (6, 2)])
+def test_matches_torch_sdpa_fp64(causal, gqa):
+    torch = pytest.importorskip("torch")
+    F = torch.nn.functional
+    S, D = 33, 16
+    Hq, Hkv = gqa
+    scale = 0.21
+    q, k, v, do = rnd((S, Hq, D), 37), rnd((S, Hkv, D), 38), rnd((S, Hkv, D), 39), rnd((S, Hq, D), 40)
+    tq = torch.tensor(q).permute(1, 0, 2)[None].requires_grad_(True)
+    tk = torch.tensor(k).permute(1, 0, 2)[None].requires_grad_(True)
+    tv = torch.tensor(v).permute(1, 0, 2)[None].requires_grad_(True)
+    to = F.scaled_dot_product_attention(tq, tk, tv, is_causal=causal, scale=scale,
+                                        enable_gqa=Hq != Hkv)
+    to.backward(torch.tensor(do).permute(1, 0, 2)[None])
+    o, lse = oracle.fwd(q, k, v, causal, scale, B=1, S=S)
+    dq, dk, dv = oracle.bwd(q, k, v, do, causal, scale, B=1, S=S)
+    np.testing.assert_allclose(o, to[0].permute(1, 0, 2).detach().numpy(), atol=1e-12)
+    np.testing.assert_allclose(dq, tq.grad[0].permute(1, 0, 2).numpy(), atol=1e-11)
+    np.testing.assert_allclose(dk, tk.grad[0].permute(1, 0, 2).numpy(), atol=1e-11)
+    np.testing.assert_allclose(dv, tv.grad[0].permute(1, 0, 2).numpy(), atol=1e-11)
+    # logsumexp against torch's own reduction of the masked score matrix
+    s = torch.einsum("qhd,khd->hqk", torch.tensor(q),
+                     torch.tensor(np.repeat(k, Hq // Hkv, axis=1))) * scale
+    if causal:
+        s = s.masked_fill(torch.triu(torch.ones(S, S, dtype=torch.bool), 1), float("-inf"))
+    np.testing.assert_allclose(lse[0], torch.logsumexp(s, -1).numpy(), atol=1e-12)
+
+
+# ---------------------------------------------------------------- row APIs
+def test_row_apis_agree_with_full():
+    lens = [70, 3, 45]
+    Hq, Hkv, D = 4, 2, 8
+    T = sum(lens)
+    cu = I.cu_seqlens_from(lens)
+    q, k, v, do = rnd((T, Hq, D), 41), rnd((T, Hkv, D), 42), rnd((T, Hkv, D), 43), rnd((T, Hq, D), 44)
+    o, lse = oracle.fwd(q, k, v, True, 0.3, cu_seqlens=cu)
+    dq, dk, dv = oracle.bwd(q, k, v, do, True, 0.3, cu_seqlens=cu)
+    rows = [(0, 1, 69), (1, 3, 2), (2, 0, 0), (2, 2, 44), (0, 0, 0)]
+    orow, lrow = oracle.fwd_rows(q, k, v, True, 0.3, rows, cu_seqlens=cu)
+    dqr, lr2, _ = oracle.bwd_dq_rows(q, k, v, do, True, 0.3, rows, cu_seqlens=cu)
+    for n, (b, h, i) in enumerate(rows):
+        t = cu[b] + i
+        assert np.array_equal(orow[n], o[t, h])
+        assert lrow[n] == lse[h, t] == lr2[n]
+        np.testing.assert_allclose(dqr[n], dq[t, h], atol=1e-13)
+    dk2, dv2 = oracle.bwd_dkdv_range(q, k, v, do, True, 0.3, b=2, g=1, j0=30, j1=45, cu_seqlens=cu)
+    np.testing.assert_allclose(dk2, dk[cu[2] + 30: cu[2] + 45, 1], atol=1e-13)
+    np.testing.assert_allclose(dv2, dv[cu[2] + 30: cu[2] + 45, 1], atol=1e-13)
+
+
+def test_rejects_bad_arguments():
+    q = np.zeros((4, 3, 2))
+    k = np.zeros((4, 2, 2))
+    with pytest.raises(ValueError):
+        oracle.fwd(q, k, k, True, 1.0, B=1, S=4)  # Hq % Hkv != 0
+    with pytest.raises(ValueError):
+        oracle.fwd(np.zeros((4, 2, 2)), k, k, True, 1.0, cu_seqlens=np.array([0, 3, 2], np.int32))
