@@ -1,0 +1,122 @@
+/*
+ * attn.h -- C ABI of libattn.so: exact scaled-dot-product attention, forward and
+ * backward, as fused tiled kernels for NVIDIA B200 (sm_100a).
+ *
+ * What is computed (page "ms-swift集成FlashAttention 2/3，长文本训练更高效"
+ * [ms-swift integrates FlashAttention 2/3]): the standard attention of section
+ * "为什么传统注意力这么'吃'显存" -- S = scale * Q K^T, a row softmax, O = P V -- computed
+ * the way section "FlashAttention 如何破局" describes: Q/K/V tiled along the
+ * sequence, an online softmax keeping a running maximum and normaliser per row,
+ * and only the output (plus the per-row log-sum-exp) written to global memory.
+ * The S x S score matrix never reaches HBM in either direction.
+ *
+ * Conventions shared by every entry point
+ *   - All tensors are row-major and contiguous, bf16 unless stated.
+ *     Dense batches (cu_seqlens == NULL): q, o, dO, dq are [B][S][Hq][D];
+ *     k, v, dk, dv are [B][S][Hkv][D]; lse is fp32 [B][Hq][S].
+ *     Packed batches (cu_seqlens != NULL): B is the number of sequences and S the
+ *     total token count T; q is [T][Hq][D], k/v [T][Hkv][D], lse [Hq][T];
+ *     cu_seqlens is a DEVICE array of B+1 int32 offsets, 0 = cu[0] <= ... <= cu[B] = T.
+ *     Sequences never attend to each other; positions count from each sequence's start.
+ *   - Grouped-query attention: query head h reads key/value head h / (Hq/Hkv).
+ *   - causal != 0 masks key j for query i when j > i (positions within the sequence).
+ *   - lse[i] = ln sum_j exp(scale * q_i . k_j) over the visible keys (natural log).
+ *   - D must be 64 or 128; Hq must be a multiple of Hkv; B, Hq, Hkv, S >= 1.
+ *   - Every tensor pointer is a device pointer owned by the caller; tensor pointers
+ *     must be 16-byte aligned (lse and cu_seqlens 4-byte aligned).
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  All work is
+ *     asynchronous on that stream; arguments are validated synchronously before
+ *     anything is launched, and nothing is launched when validation fails.
+ *   - The library allocates no device memory and keeps no per-call state.
+ *   - A packed batch whose cu_seqlens break the rules above cannot make a kernel read
+ *     or write outside the tensors (every sequence is clamped to [0, T)), but its
+ *     results are undefined; attn_check_cu_seqlens validates a host copy.
+ *   - Device-side waits are bounded; a wait that times out makes the kernel skip
+ *     its remaining work and records the event in a sticky status word that
+ *     attn_device_status reports.
+ */
+#ifndef ATTN_H_
+#define ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ATTN_OK = 0,
+  ATTN_ERR_INVALID_ARG = 1,   /* bad size, null pointer, Hq % Hkv != 0, scale not finite,
+                                 workspace too small, malformed host cu_seqlens */
+  ATTN_ERR_UNSUPPORTED = 2,   /* D not in {64, 128}, or the device is not sm_100 */
+  ATTN_ERR_MISALIGNED = 3,    /* a pointer breaks the alignment rules above */
+  ATTN_ERR_CUDA = 4,          /* a CUDA runtime/driver call or a launch failed */
+  ATTN_ERR_TIMEOUT = 5        /* a device-side bounded wait gave up (see attn_device_status) */
+} attn_status;
+
+/* Forward pass (page section "FlashAttention 如何破局": tiled QK^T -> online softmax -> PV).
+ * Writes o (same layout as q) and lse. */
+attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                     int Hq, int Hkv, int S, int D, int causal, float scale,
+                     const int32_t* cu_seqlens, void* stream);
+
+/* Bytes of device workspace attn_bwd needs for these arguments (same meaning as in
+ * attn_bwd; only whether cu_seqlens is NULL matters).  Holds the fp32 dQ accumulator
+ * [T][Hq][D], and Delta = rowsum(dO * O) and LSE*log2(e) in 128-row tiles.
+ * Returns 0 for invalid sizes. */
+size_t attn_bwd_workspace_size(int B, int Hq, int S, int D, const int32_t* cu_seqlens);
+
+/* Backward pass (page section "为什么传统注意力这么'吃'显存": the intermediates are
+ * recomputed, not stored -- P is rebuilt tile by tile from lse).
+ * Inputs q, k, v, o, lse (from attn_fwd with the same arguments) and dout = dL/dO;
+ * outputs dq, dk, dv (layouts of q, k, v).  dk/dv are summed over the query heads of
+ * each group.  `workspace` (>= attn_bwd_workspace_size bytes, 256-byte aligned) is
+ * scratch owned by the caller; its contents need no initialisation.
+ * dq is accumulated with fp32 atomics, so its last bits can differ run to run;
+ * o, lse, dk and dv are deterministic. */
+attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o,
+                     const float* lse, const void* dout, void* dq, void* dk, void* dv, int B,
+                     int Hq, int Hkv, int S, int D, int causal, float scale,
+                     const int32_t* cu_seqlens, void* workspace, size_t workspace_bytes,
+                     void* stream);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* attn_strerror(attn_status status);
+
+/* Synchronises `stream`, then returns ATTN_ERR_TIMEOUT if any kernel of this library
+ * recorded a timed-out wait on the current device since the last call (and clears
+ * the record), ATTN_ERR_CUDA if the stream reports a CUDA error, else ATTN_OK.
+ * If `site` is not NULL it receives the code of the first wait that timed out. */
+attn_status attn_device_status(void* stream, unsigned* site);
+
+/* Sets the limit of every device-side wait, in nanoseconds (default 2e9). */
+void attn_set_wait_timeout_ns(unsigned long long ns);
+
+/* Validates a HOST copy of cu_seqlens: B+1 entries, cu[0] = 0, non-decreasing,
+ * cu[B] = S.  Returns ATTN_OK or ATTN_ERR_INVALID_ARG. */
+attn_status attn_check_cu_seqlens(const int32_t* cu_host, int B, int S);
+
+/* Self-test of the failure path: launches one CTA that waits on a barrier nobody
+ * arrives on, with a limit of `timeout_ns`.  The wait must give up and record a
+ * timeout; call attn_device_status afterwards to observe it.  No page counterpart:
+ * it exists to test the bounded-wait machinery without faulting the GPU. */
+attn_status attn_selftest_wait_timeout(unsigned long long timeout_ns, void* stream);
+
+/* Self-test of the tensor-core operand layouts (no page counterpart).  One 128-row
+ * tile, D in {64, 128}; a, b, p, at, c are device pointers:
+ *   mode 0: c[128][128] = a[128][D] . b[128][D]^T          (a, b bf16)
+ *   mode 1: c[128][D]   = bf16(p[128][128]) . b[128][D]    (p fp32, b bf16)
+ *   mode 2: c[128][D]   = at[128][128]^T . b[128][D]       (at, b bf16)
+ * c is fp32. */
+attn_status attn_selftest_umma(int mode, int D, const void* a, const void* b, const float* p,
+                               const void* at, float* c, void* stream);
+
+/* Library ABI version (major*100 + minor). */
+int attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_H_ */

@@ -1,0 +1,498 @@
+// attn_bwd.cuh -- fused attention backward for sm_100a.
+//
+// The page "ms-swift集成FlashAttention 2/3" (section "为什么传统注意力这么'吃'显存",
+// why standard attention eats so much memory) notes that the backward pass of the
+// native implementation needs the S x S intermediates again, cached or recomputed;
+// the fused kernel (section "FlashAttention 如何破局") keeps none of them in HBM.
+// Here the backward recomputes the probabilities tile by tile from the per-row
+// log-sum-exp the forward saved:
+//     P = exp(scale * Q K^T - LSE),  dP = dO V^T,  Delta = rowsum(dO * O),
+//     dS = P * (dP - Delta),  dV = P^T dO,  dK = scale dS^T Q,  dQ = scale dS K.
+//
+// Kernels:
+//   bwd_preprocess  Delta and LSE*log2(e) per query row into a tile-padded workspace
+//                   (rows past a sequence end get LSE = +inf, so their P is exactly 0),
+//                   and zeroes the fp32 dQ accumulator rows.
+//   attn_bwd_kernel KV-stationary: one CTA holds a 128-key tile of one kv head (K, V in
+//                   shared memory, dK/dV accumulators in TMEM) and loops over the query
+//                   heads of its group and the 128-row query tiles that see it.
+//                   Per query tile: S^T = K Q^T, dP^T = V dO^T, dV += P^T dO,
+//                   dK += dS^T Q (P^T, dS^T read from TMEM as bf16), dQ_tile = dS K
+//                   (dS staged in shared memory), and dQ_tile is reduced into the fp32
+//                   accumulator with vector atomics.  dK/dV stay deterministic.
+//   dq_convert      dq = bf16(scale * accumulator).
+//
+// Warps: 0-3 compute P^T and dS^T (one thread per key row), 4-7 drain dQ from TMEM
+// into the accumulator, 8 is the TMA producer, 9 issues the MMAs.
+#pragma once
+#include <cuda_bf16.h>
+#include "attn_common.cuh"
+#include "sm100_ptx.cuh"
+
+namespace attn_sm100 {
+namespace bwd {
+
+constexpr int kThreads = 320;
+constexpr int kWarpTMA = 8;
+constexpr int kWarpMMA = 9;
+constexpr int kSlab = 128 * 128;
+
+struct Params {
+  SeqView sv;
+  float* dq_acc;          // [T][Hq][D] fp32
+  const float* lse2;      // [Hq][ntile][128]
+  const float* delta;     // [Hq][ntile][128]
+  __nv_bfloat16* dk;      // [T][Hkv][D]
+  __nv_bfloat16* dv;
+  int Hq, Hkv, G, T, causal;
+  int ntile;              // tiles per head in the lse2/delta workspace
+  int nkv;                // (T >> 7) + nseq: upper bound of 128-key blocks
+  float scale_log2;
+  float scale;
+  unsigned* status;
+  unsigned long long timeout_ns;
+};
+
+template <int D>
+struct Cfg {
+  static constexpr int TILE = 128 * D * 2;  // one 128-row bf16 tile
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = OFF_K + TILE;
+  static constexpr int OFF_Q = OFF_V + TILE;        // 2 stages
+  static constexpr int OFF_DO = OFF_Q + 2 * TILE;   // 2 stages
+  static constexpr int OFF_DS = OFF_DO + 2 * TILE;  // 128 x 128 bf16, MN-major for the dQ MMA
+  static constexpr int OFF_LSE = OFF_DS + 128 * 128 * 2;  // 2 stages x 128 fp32
+  static constexpr int OFF_DELTA = OFF_LSE + 2 * 512;
+  static constexpr int OFF_BAR = OFF_DELTA + 2 * 512;
+  // kv_full, q_full[2], q_empty[2], s_full, dp_full, p_full, ds_full, dq_full, dq_free, dkv_final, drain
+  static constexpr int NBAR = 13;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16;
+  static constexpr int kMaxDyn = 232448;
+  static constexpr int SLACK = (SMEM_BYTES + 1024 <= kMaxDyn) ? 1024 : (kMaxDyn - SMEM_BYTES);
+  static constexpr int SMEM_ALLOC = SMEM_BYTES + SLACK;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DQ = 128, COL_DV = 256, COL_DK = 256 + D;
+  static_assert(SMEM_BYTES <= kMaxDyn, "shared memory budget");
+};
+
+enum : unsigned {
+  kSiteKV = 0x200, kSiteQEmpty, kSiteQFull, kSiteSFull, kSiteDpFull, kSitePFull, kSiteDsFull,
+  kSiteDqFull, kSiteDqFree, kSiteFinal
+};
+
+// ---------------------------------------------------------------- preprocess
+// grid (nkv, Hq), 128 threads: one thread per query row of one 128-row tile.
+template <int D>
+__global__ void __launch_bounds__(128)
+bwd_preprocess_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
+                      const float* __restrict__ lse, float* __restrict__ lse2,
+                      float* __restrict__ delta, float* __restrict__ dq_acc, SeqView sv, int Hq,
+                      int T, int ntile) {
+  int seq, m, start, len;
+  if (!locate_block<7>(sv, blockIdx.x, seq, m, start, len)) return;
+  const int h = blockIdx.y;
+  const int r = threadIdx.x;
+  const int qpos = m * 128 + r;
+  float dl = 0.f, l2 = INFINITY;
+  if (qpos < len) {
+    const size_t row = (size_t(start + qpos) * Hq + h) * D;
+    const uint4* po = reinterpret_cast<const uint4*>(o + row);
+    const uint4* pd = reinterpret_cast<const uint4*>(dout + row);
+    float acc = 0.f;
+#pragma unroll 4
+    for (int i = 0; i < D / 8; ++i) {
+      const uint4 a = __ldg(po + i), b = __ldg(pd + i);
+      const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
+      const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&b);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float2 fa = __bfloat1622float2(a2[k]);
+        const float2 fb = __bfloat1622float2(b2[k]);
+        acc = fmaf(fa.x, fb.x, acc);
+        acc = fmaf(fa.y, fb.y, acc);
+      }
+    }
+    dl = acc;
+    const size_t li = sv.cu ? size_t(h) * T + start + qpos : (size_t(seq) * Hq + h) * sv.S + qpos;
+    l2 = lse[li] * 1.4426950408889634f;
+    float4* z = reinterpret_cast<float4*>(dq_acc + row);
+#pragma unroll 4
+    for (int i = 0; i < D / 4; ++i) z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  const size_t wi = (size_t(h) * ntile + blockIdx.x) * 128 + r;
+  lse2[wi] = l2;
+  delta[wi] = dl;
+}
+
+// ---------------------------------------------------------------- dq convert
+__global__ void __launch_bounds__(256)
+dq_convert_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ dq, size_t n8,
+                  float scale) {
+  for (size_t i = blockIdx.x * size_t(blockDim.x) + threadIdx.x; i < n8;
+       i += size_t(gridDim.x) * blockDim.x) {
+    const float4 a = __ldg(reinterpret_cast<const float4*>(acc) + 2 * i);
+    const float4 b = __ldg(reinterpret_cast<const float4*>(acc) + 2 * i + 1);
+    uint4 out;
+    out.x = pack_bf16x2(a.x * scale, a.y * scale);
+    out.y = pack_bf16x2(a.z * scale, a.w * scale);
+    out.z = pack_bf16x2(b.x * scale, b.y * scale);
+    out.w = pack_bf16x2(b.z * scale, b.w * scale);
+    reinterpret_cast<uint4*>(dq)[i] = out;
+  }
+}
+
+// ---------------------------------------------------------------- main kernel
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                const Params p) {
+  using C = Cfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+  if (pad > uint32_t(C::SLACK)) {
+    if (threadIdx.x == 0) atomicOr(p.status, kStatusSmemAlign);
+    return;
+  }
+  uint8_t* smem = smem_raw + pad;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- work item: (sequence, kv head, 128-key tile); low tiles (most query tiles) first.
+  const int g = blockIdx.x % p.Hkv;
+  int seq, n, start, len;
+  if (!locate_block<7>(p.sv, int(blockIdx.x / p.Hkv), seq, n, start, len)) return;
+  const int nq = (len + 127) >> 7;
+  const int m0 = p.causal ? n : 0;
+  const int per_head = nq - m0;
+  const int iters = p.G * per_head;
+  const int tile_base = (start >> 7) + seq;  // workspace tile index of query tile 0
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* kv_full = bars;
+  uint64_t* q_full = bars + 1;
+  uint64_t* q_empty = bars + 3;
+  uint64_t* s_full = bars + 5;
+  uint64_t* dp_full = bars + 6;
+  uint64_t* p_full = bars + 7;
+  uint64_t* ds_full = bars + 8;
+  uint64_t* dq_full = bars + 9;
+  uint64_t* dq_free = bars + 10;
+  uint64_t* dkv_final = bars + 11;
+  uint64_t* drain = bars + 12;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+  float* lse_s = reinterpret_cast<float*>(smem + C::OFF_LSE);
+  float* delta_s = reinterpret_cast<float*>(smem + C::OFF_DELTA);
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    mbar_init(kv_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(dp_full, 1);
+    mbar_init(p_full, 4);
+    mbar_init(ds_full, 4);
+    mbar_init(dq_full, 1);
+    mbar_init(dq_free, 4);
+    mbar_init(dkv_final, 1);
+    mbar_init(drain, 1);
+    fence_mbar_init();
+  }
+  if (warp == kWarpMMA) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == kWarpTMA && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(&tm_do);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const WaitCtl wc{p.status, abort_flag, p.timeout_ns};
+
+  if (warp == kWarpTMA) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int nissued = 0;
+      mbar_arrive_expect_tx(kv_full, 2 * C::TILE);
+      for (int hf = 0; hf < D / 64; ++hf) {
+        tma_load_3d(&tm_k, kv_full, smem + C::OFF_K + hf * kSlab, hf * 64, g, start + 128 * n);
+        tma_load_3d(&tm_v, kv_full, smem + C::OFF_V + hf * kSlab, hf * 64, g, start + 128 * n);
+      }
+      for (int it = 0; it < iters; ++it) {
+        const int st = it & 1;
+        const int hq = g * p.G + it / per_head;
+        const int m = m0 + it % per_head;
+        if (!mbar_wait(&q_empty[st], ((it >> 1) & 1) ^ 1, wc, kSiteQEmpty)) break;
+        mbar_arrive_expect_tx(&q_full[st], 2 * C::TILE + 1024);
+        for (int hf = 0; hf < D / 64; ++hf) {
+          tma_load_3d(&tm_q, &q_full[st], smem + C::OFF_Q + st * C::TILE + hf * kSlab, hf * 64, hq,
+                      start + 128 * m);
+          tma_load_3d(&tm_do, &q_full[st], smem + C::OFF_DO + st * C::TILE + hf * kSlab, hf * 64,
+                      hq, start + 128 * m);
+        }
+        const size_t wi = (size_t(hq) * p.ntile + tile_base + m) * 128;
+        bulk_load(lse_s + st * 128, p.lse2 + wi, 512, &q_full[st]);
+        bulk_load(delta_s + st * 128, p.delta + wi, 512, &q_full[st]);
+        ++nissued;
+      }
+      mbar_drain(kv_full, 0, drain_ns(abort_flag, p.timeout_ns));
+      for (int st = 0; st < 2; ++st) {
+        const int c = nissued > st ? (nissued - 1 - st) / 2 + 1 : 0;
+        if (c) mbar_drain(&q_full[st], (c - 1) & 1, drain_ns(abort_flag, p.timeout_ns));
+      }
+    }
+  } else if (warp == kWarpMMA) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16_f32(128, 128, 0, 0);   // S^T, dP^T
+      constexpr uint32_t idKV = idesc_bf16_f32(128, D, 0, 1);    // dV, dK (A from TMEM)
+      constexpr uint32_t idQ = idesc_bf16_f32(128, D, 1, 1);     // dQ (A = dS, MN-major)
+      const uint32_t kb = smem_u32(smem + C::OFF_K);
+      const uint32_t vb = smem_u32(smem + C::OFF_V);
+      const uint32_t dsb = smem_u32(smem + C::OFF_DS);
+      auto issue_T = [&](uint32_t col, uint32_t ab, uint32_t bb) {  // [128 x 128] = A B^T over D
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * kSlab + (kk & 3) * 32;
+          mma_ss(tmem + col, sdesc_sw128(ab + off, 16, 1024), sdesc_sw128(bb + off, 16, 1024), idS,
+                 kk > 0 ? 1u : 0u);
+        }
+      };
+      bool ok = mbar_wait(kv_full, 0, wc, kSiteKV) && mbar_wait(&q_full[0], 0, wc, kSiteQFull);
+      if (ok && iters > 0) {
+        tc_fence_after();
+        issue_T(C::COL_S, kb, smem_u32(smem + C::OFF_Q));
+        mma_commit(s_full);
+      }
+      for (int it = 0; it < iters && ok; ++it) {
+        const int st = it & 1;
+        const uint32_t qb = smem_u32(smem + C::OFF_Q + st * C::TILE);
+        const uint32_t dob = smem_u32(smem + C::OFF_DO + st * C::TILE);
+        if (it > 0 && !(ok = mbar_wait(dq_free, (it - 1) & 1, wc, kSiteDqFree))) break;
+        tc_fence_after();
+        issue_T(C::COL_DP, vb, dob);  // dP^T = V dO^T
+        mma_commit(dp_full);
+        if (!(ok = mbar_wait(p_full, it & 1, wc, kSitePFull))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)  // dV += P^T dO
+          mma_ts(tmem + C::COL_DV, tmem + C::COL_S + kk * 8, sdesc_sw128(dob + kk * 2048, kSlab, 1024),
+                 idKV, (it > 0 || kk > 0) ? 1u : 0u);
+        if (it + 1 < iters) {
+          if (!(ok = mbar_wait(&q_full[st ^ 1], ((it + 1) >> 1) & 1, wc, kSiteQFull))) break;
+          tc_fence_after();
+          issue_T(C::COL_S, kb, smem_u32(smem + C::OFF_Q + (st ^ 1) * C::TILE));  // next S^T
+          mma_commit(s_full);
+        }
+        if (!(ok = mbar_wait(ds_full, it & 1, wc, kSiteDsFull))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)  // dK += dS^T Q
+          mma_ts(tmem + C::COL_DK, tmem + C::COL_DP + kk * 8, sdesc_sw128(qb + kk * 2048, kSlab, 1024),
+                 idKV, (it > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)  // dQ_tile = dS K
+          mma_ss(tmem + C::COL_DQ, sdesc_sw128(dsb + kk * 2048, 16384, 1024),
+                 sdesc_sw128(kb + kk * 2048, kSlab, 1024), idQ, kk > 0 ? 1u : 0u);
+        mma_commit(dq_full);
+        mma_commit(&q_empty[st]);
+      }
+      if (ok) mma_commit(dkv_final);
+      mma_commit(drain);
+      mbar_drain(drain, 0, drain_ns(abort_flag, p.timeout_ns));
+    }
+  } else if (warp < 4) {
+    // ------------------------------------------------------------ P^T and dS^T
+    const int qw = warp;
+    const int r = qw * 32 + lane;      // key row in the tile
+    const int kpos = n * 128 + r;
+    const bool key_ok = p.causal || kpos < len;
+    const float c = p.scale_log2;
+    const uint32_t tS = tmem_addr(tmem, qw * 32, C::COL_S);
+    const uint32_t tP = tmem_addr(tmem, qw * 32, C::COL_DP);
+    uint8_t* ds_row = smem + C::OFF_DS + (r >> 3) * 1024 + (r & 7) * 128;
+    bool ok = true;
+    for (int it = 0; it < iters; ++it) {
+      const int st = it & 1;
+      const int m = m0 + it % per_head;
+      ok = __all_sync(0xffffffffu, mbar_wait(s_full, it & 1, wc, kSiteSFull) &&
+                                       mbar_wait(&q_full[st], (it >> 1) & 1, wc, kSiteQFull));
+      if (!ok) break;
+      tc_fence_after();
+      const float* lse_t = lse_s + st * 128;
+      const float* dlt_t = delta_s + st * 128;
+      float pr[128];
+      {
+        uint32_t u0[32], u1[32], u2[32], u3[32];
+        tmem_ld32(tS + 0, u0);
+        tmem_ld32(tS + 32, u1);
+        tmem_ld32(tS + 64, u2);
+        tmem_ld32(tS + 96, u3);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          pr[i] = __uint_as_float(u0[i]);
+          pr[32 + i] = __uint_as_float(u1[i]);
+          pr[64 + i] = __uint_as_float(u2[i]);
+          pr[96 + i] = __uint_as_float(u3[i]);
+        }
+      }
+      const bool diag = p.causal && m == n;
+#pragma unroll
+      for (int i = 0; i < 128; ++i) {
+        const float e = ex2_approx(fmaf(pr[i], c, -lse_t[i]));
+        pr[i] = (key_ok && !(diag && i < r)) ? e : 0.f;
+      }
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(pr[ch * 32 + 2 * i], pr[ch * 32 + 2 * i + 1]);
+        tmem_st16(tS + ch * 16, pk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full);
+
+      // dS^T = P^T * (dP^T - Delta): written in place into the dP columns (bf16) for the
+      // dK MMA and into shared memory (MN-major) for the dQ MMA.
+      ok = __all_sync(0xffffffffu, mbar_wait(dp_full, it & 1, wc, kSiteDpFull) &&
+                                       (it == 0 || mbar_wait(dq_full, (it - 1) & 1, wc, kSiteDqFull)));
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t u[32];
+        tmem_ld32(tP + ch * 32, u);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int c0 = ch * 32 + 2 * i;
+          const float d0 = pr[c0] * (__uint_as_float(u[2 * i]) - dlt_t[c0]);
+          const float d1 = pr[c0 + 1] * (__uint_as_float(u[2 * i + 1]) - dlt_t[c0 + 1]);
+          pk[i] = pack_bf16x2(d0, d1);
+        }
+        tmem_st16(tP + ch * 16, pk);
+        // shared memory: query rows ch*32 .. ch*32+31 -> 64-row block ch/2, 16-byte chunks
+        uint8_t* blk = ds_row + (ch >> 1) * 16384;
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const int chunk = (ch & 1) * 4 + q4;
+          *reinterpret_cast<uint4*>(blk + ((chunk ^ (r & 7)) << 4)) =
+              make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+        }
+      }
+      fence_async_smem();
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(ds_full);
+    }
+    // epilogue: dV rows
+    if (ok) {
+      ok = __all_sync(0xffffffffu, mbar_wait(dkv_final, 0, wc, kSiteFinal));
+      if (ok) {
+        tc_fence_after();
+        const uint32_t tV = tmem_addr(tmem, qw * 32, C::COL_DV);
+        __nv_bfloat16* dst = p.dv + (size_t(start + kpos) * p.Hkv + g) * D;
+#pragma unroll 1
+        for (int ch = 0; ch < D / 32; ++ch) {
+          uint32_t u[32];
+          tmem_ld32(tV + ch * 32, u);
+          tmem_wait_ld();
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            pk[i] = pack_bf16x2(__uint_as_float(u[2 * i]), __uint_as_float(u[2 * i + 1]));
+          if (kpos < len) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst + ch * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              d4[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+          }
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ dQ drain (warps 4-7)
+    const int qw = warp & 3;
+    const int r = qw * 32 + lane;      // query row of the tile (dQ) / key row (dK epilogue)
+    const uint32_t tQ = tmem_addr(tmem, qw * 32, C::COL_DQ);
+    bool ok = true;
+    for (int it = 0; it < iters; ++it) {
+      const int hq = g * p.G + it / per_head;
+      const int m = m0 + it % per_head;
+      ok = __all_sync(0xffffffffu, mbar_wait(dq_full, it & 1, wc, kSiteDqFull));
+      if (!ok) break;
+      tc_fence_after();
+      float acc[D];
+#pragma unroll
+      for (int ch = 0; ch < D / 32; ++ch) {
+        uint32_t u[32];
+        tmem_ld32(tQ + ch * 32, u);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) acc[ch * 32 + i] = __uint_as_float(u[i]);
+      }
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(dq_free);
+      const int qpos = m * 128 + r;
+      if (qpos < len) {
+        float4* dst = reinterpret_cast<float4*>(p.dq_acc + (size_t(start + qpos) * p.Hq + hq) * D);
+#pragma unroll
+        for (int i = 0; i < D / 4; ++i)
+          atomicAdd(dst + i, make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]));
+      }
+    }
+    // epilogue: dK rows (scaled)
+    if (ok) {
+      ok = __all_sync(0xffffffffu, mbar_wait(dkv_final, 0, wc, kSiteFinal));
+      if (ok) {
+        tc_fence_after();
+        const int kpos = n * 128 + r;
+        const uint32_t tK = tmem_addr(tmem, qw * 32, C::COL_DK);
+        __nv_bfloat16* dst = p.dk + (size_t(start + kpos) * p.Hkv + g) * D;
+#pragma unroll 1
+        for (int ch = 0; ch < D / 32; ++ch) {
+          uint32_t u[32];
+          tmem_ld32(tK + ch * 32, u);
+          tmem_wait_ld();
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            pk[i] = pack_bf16x2(__uint_as_float(u[2 * i]) * p.scale,
+                                __uint_as_float(u[2 * i + 1]) * p.scale);
+          if (kpos < len) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst + ch * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              d4[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kWarpMMA) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+}  // namespace bwd
+}  // namespace attn_sm100

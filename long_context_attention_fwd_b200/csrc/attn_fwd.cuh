@@ -1,0 +1,382 @@
+// attn_fwd.cuh -- fused attention forward for sm_100a.
+//
+// Follows the fused, tiled scheme of the page "ms-swift集成FlashAttention 2/3，长文本训练更高效"
+// [ms-swift integrates FlashAttention 2/3], section "FlashAttention 如何破局"
+// [how FlashAttention breaks the deadlock]: Q, K, V are cut into tiles along the
+// sequence, a block holds its Q tile and streams the K/V tiles of the same sequence
+// through on-chip memory, runs QK^T -> softmax -> PV there with an online softmax
+// (running maximum and normaliser per row), and writes only the output (plus the
+// row log-sum-exp kept for the backward pass).
+//
+// Blackwell mapping (one CTA = 256 query rows of one head, as two 128-row tiles):
+//   warp 8      TMA producer: Q tiles once, then K_j / V_j into a ring of NS stages.
+//   warp 9      MMA issuer (one thread): S_t = Q_t K_j^T (SS, fp32 in TMEM) and
+//               O_t += P_t V_j (P read from TMEM as bf16, V from shared memory).
+//   warps 0-3   softmax for tile 0, warps 4-7 for tile 1: one thread per query row,
+//               reads S from TMEM, exp2-based online max/sum, writes P (bf16) back
+//               into the S columns, rescales O in TMEM when the running max grows by
+//               more than 2^8, and finally normalises O and stores O and LSE.
+// The two tiles ping-pong: while softmax works on one tile the tensor core runs the
+// other tile's PV and the next S, so MMA and exponentials overlap.
+#pragma once
+#include <cuda_bf16.h>
+#include "attn_common.cuh"
+#include "sm100_ptx.cuh"
+
+namespace attn_sm100 {
+namespace fwd {
+
+constexpr int BM = 128;                // query rows per tile
+constexpr int BN = 128;                // keys per K/V tile
+constexpr int kThreads = 320;          // 10 warps
+constexpr int kWarpTMA = 8;
+constexpr int kWarpMMA = 9;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when max grows > 2^8
+constexpr int kSlab = 128 * 128;       // one 128-row x 64-column bf16 swizzled slab (16 KB)
+
+struct Params {
+  SeqView sv;
+  __nv_bfloat16* o;
+  float* lse;
+  int Hq, G, T;                        // query heads, query heads per kv head, total tokens
+  int causal;
+  float scale_log2;                    // softmax scale * log2(e)
+  int nblk;                            // (T >> 8) + nseq: upper bound of 256-row blocks
+  unsigned* status;
+  unsigned long long timeout_ns;
+};
+
+template <int D>
+struct Cfg {
+  static constexpr int NS = (D == 128) ? 2 : 4;
+  static constexpr int QT_BYTES = BM * D * 2;
+  static constexpr int KV_BYTES = BN * D * 2;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + 2 * QT_BYTES;
+  static constexpr int OFF_V = OFF_K + NS * KV_BYTES;
+  static constexpr int OFF_BAR = OFF_V + NS * KV_BYTES;
+  // q_full, k_full[NS], k_empty[NS], v_full[NS], v_empty[NS], s_full[2], p_full[2], o_final[2], drain
+  static constexpr int NBAR = 1 + 4 * NS + 7;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16;
+  static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;  // slack for 1024-byte alignment
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O0 = 256, COL_O1 = 256 + D;
+};
+
+// Wait-site codes reported in the status word when a wait times out.
+enum : unsigned {
+  kSiteKEmpty = 0x100, kSiteVEmpty, kSiteQFull, kSiteKFull, kSiteVFull, kSitePFull, kSiteSFull,
+  kSiteOFinal
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const Params p) {
+  using C = Cfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- work item: (sequence, head, 256-row block), longest causal blocks first.
+  const int h = blockIdx.x % p.Hq;
+  const int gblk = p.nblk - 1 - int(blockIdx.x / p.Hq);
+  int seq, mb, start, len;
+  if (!locate_block<8>(p.sv, gblk, seq, mb, start, len)) return;  // uniform: no work
+  const int g = h / p.G;
+  const int q_row0 = mb * 256;
+  int n_t[2];
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const int r0 = q_row0 + BM * t;
+    if (r0 >= len) n_t[t] = 0;
+    else if (p.causal) n_t[t] = (min(r0 + BM - 1, len - 1) >> 7) + 1;
+    else n_t[t] = (len + BN - 1) >> 7;
+  }
+  const int jmax = max(n_t[0], n_t[1]);
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* q_full = bars;
+  uint64_t* k_full = bars + 1;
+  uint64_t* k_empty = k_full + C::NS;
+  uint64_t* v_full = k_empty + C::NS;
+  uint64_t* v_empty = v_full + C::NS;
+  uint64_t* s_full = v_empty + C::NS;
+  uint64_t* p_full = s_full + 2;
+  uint64_t* o_final = p_full + 2;
+  uint64_t* drain = o_final + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    mbar_init(q_full, 1);
+    for (int i = 0; i < C::NS; ++i) {
+      mbar_init(&k_full[i], 1);
+      mbar_init(&k_empty[i], 1);
+      mbar_init(&v_full[i], 1);
+      mbar_init(&v_empty[i], 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&s_full[t], 1);
+      mbar_init(&p_full[t], 4);
+      mbar_init(&o_final[t], 1);
+    }
+    mbar_init(drain, 1);
+    fence_mbar_init();
+  }
+  if (warp == kWarpMMA) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == kWarpTMA && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const WaitCtl wc{p.status, abort_flag, p.timeout_ns};
+
+  if (warp == kWarpTMA) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int nk = 0, nv = 0;
+      const uint32_t qbytes = (n_t[0] > 0 ? C::QT_BYTES : 0) + (n_t[1] > 0 ? C::QT_BYTES : 0);
+      mbar_arrive_expect_tx(q_full, qbytes);
+      for (int t = 0; t < 2; ++t) {
+        if (n_t[t] == 0) continue;
+        for (int hf = 0; hf < D / 64; ++hf)
+          tma_load_3d(&tm_q, q_full, smem + C::OFF_Q + t * C::QT_BYTES + hf * kSlab, hf * 64, h,
+                      start + q_row0 + BM * t);
+      }
+      for (int j = 0; j < jmax; ++j) {
+        const int st = j % C::NS;
+        const uint32_t ph = (j / C::NS) & 1;
+        if (!mbar_wait(&k_empty[st], ph ^ 1, wc, kSiteKEmpty)) break;
+        mbar_arrive_expect_tx(&k_full[st], C::KV_BYTES);
+        for (int hf = 0; hf < D / 64; ++hf)
+          tma_load_3d(&tm_k, &k_full[st], smem + C::OFF_K + st * C::KV_BYTES + hf * kSlab,
+                      hf * 64, g, start + BN * j);
+        ++nk;
+        if (!mbar_wait(&v_empty[st], ph ^ 1, wc, kSiteVEmpty)) break;
+        mbar_arrive_expect_tx(&v_full[st], C::KV_BYTES);
+        for (int hf = 0; hf < D / 64; ++hf)
+          tma_load_3d(&tm_v, &v_full[st], smem + C::OFF_V + st * C::KV_BYTES + hf * kSlab,
+                      hf * 64, g, start + BN * j);
+        ++nv;
+      }
+      // Drain: every issued copy must land before shared memory is released.
+      mbar_drain(q_full, 0, drain_ns(abort_flag, p.timeout_ns));
+      for (int st = 0; st < C::NS; ++st) {
+        const int ck = nk > st ? (nk - 1 - st) / C::NS + 1 : 0;
+        const int cv = nv > st ? (nv - 1 - st) / C::NS + 1 : 0;
+        if (ck) mbar_drain(&k_full[st], (ck - 1) & 1, drain_ns(abort_flag, p.timeout_ns));
+        if (cv) mbar_drain(&v_full[st], (cv - 1) & 1, drain_ns(abort_flag, p.timeout_ns));
+      }
+    }
+  } else if (warp == kWarpMMA) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16_f32(128, 128, 0, 0);
+      constexpr uint32_t idPV = idesc_bf16_f32(128, D, 0, 1);
+      const uint32_t qb[2] = {smem_u32(smem + C::OFF_Q), smem_u32(smem + C::OFF_Q + C::QT_BYTES)};
+      const uint32_t colS[2] = {C::COL_S0, C::COL_S1};
+      const uint32_t colO[2] = {C::COL_O0, C::COL_O1};
+      auto issue_S = [&](int t, int st) {
+        const uint32_t kb = smem_u32(smem + C::OFF_K + st * C::KV_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * kSlab + (kk & 3) * 32;
+          mma_ss(tmem + colS[t], sdesc_sw128(qb[t] + off, 16, 1024),
+                 sdesc_sw128(kb + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_PV = [&](int t, int st, bool acc) {
+        const uint32_t vb = smem_u32(smem + C::OFF_V + st * C::KV_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk)
+          mma_ts(tmem + colO[t], tmem + colS[t] + kk * 8, sdesc_sw128(vb + kk * 2048, kSlab, 1024),
+                 idPV, (acc || kk > 0) ? 1u : 0u);
+      };
+      bool ok = mbar_wait(q_full, 0, wc, kSiteQFull) && mbar_wait(&k_full[0], 0, wc, kSiteKFull);
+      if (ok) {
+        tc_fence_after();
+        for (int t = 0; t < 2; ++t)
+          if (n_t[t] > 0) {
+            issue_S(t, 0);
+            mma_commit(&s_full[t]);
+          }
+        mma_commit(&k_empty[0]);
+        for (int j = 0; j < jmax && ok; ++j) {
+          const int st = j % C::NS;
+          if (!(ok = mbar_wait(&v_full[st], (j / C::NS) & 1, wc, kSiteVFull))) break;
+          tc_fence_after();
+          if (j < n_t[0]) {
+            if (!(ok = mbar_wait(&p_full[0], j & 1, wc, kSitePFull))) break;
+            tc_fence_after();
+            issue_PV(0, st, j > 0);
+            if (j == n_t[0] - 1) mma_commit(&o_final[0]);
+          }
+          const bool nxt = j + 1 < jmax;
+          const int st1 = (j + 1) % C::NS;
+          if (nxt) {
+            if (!(ok = mbar_wait(&k_full[st1], ((j + 1) / C::NS) & 1, wc, kSiteKFull))) break;
+            tc_fence_after();
+            if (j + 1 < n_t[0]) {
+              issue_S(0, st1);
+              mma_commit(&s_full[0]);
+            }
+          }
+          if (j < n_t[1]) {
+            if (!(ok = mbar_wait(&p_full[1], j & 1, wc, kSitePFull))) break;
+            tc_fence_after();
+            issue_PV(1, st, j > 0);
+            if (j == n_t[1] - 1) mma_commit(&o_final[1]);
+          }
+          mma_commit(&v_empty[st]);
+          if (nxt) {
+            if (j + 1 < n_t[1]) {
+              issue_S(1, st1);
+              mma_commit(&s_full[1]);
+            }
+            mma_commit(&k_empty[st1]);
+          }
+        }
+      }
+      // Drain: all MMAs must finish before TMEM and shared memory are released.
+      mma_commit(drain);
+      mbar_drain(drain, 0, drain_ns(abort_flag, p.timeout_ns));
+    }
+  } else {
+    // ------------------------------------------------------------ softmax + epilogue
+    const int t = warp >> 2;
+    const int qw = warp & 3;
+    const int r = qw * 32 + lane;
+    const int rpos = q_row0 + BM * t + r;
+    const int n = n_t[t];
+    const float c = p.scale_log2;
+    const uint32_t colS = t ? C::COL_S1 : C::COL_S0;
+    const uint32_t colO = t ? C::COL_O1 : C::COL_O0;
+    const uint32_t tS = tmem_addr(tmem, qw * 32, colS);
+    const uint32_t tO = tmem_addr(tmem, qw * 32, colO);
+    float m_run = -INFINITY;  // reference maximum (log2 units) the accumulator is scaled to
+    float l_run = 0.f;        // running normaliser relative to m_run
+    bool ok = true;
+    for (int j = 0; j < n; ++j) {
+      ok = __all_sync(0xffffffffu, mbar_wait(&s_full[t], j & 1, wc, kSiteSFull));
+      if (!ok) break;
+      tc_fence_after();
+      float s[128];
+      {
+        uint32_t u0[32], u1[32], u2[32], u3[32];
+        tmem_ld32(tS + 0, u0);
+        tmem_ld32(tS + 32, u1);
+        tmem_ld32(tS + 64, u2);
+        tmem_ld32(tS + 96, u3);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          s[i] = __uint_as_float(u0[i]);
+          s[32 + i] = __uint_as_float(u1[i]);
+          s[64 + i] = __uint_as_float(u2[i]);
+          s[96 + i] = __uint_as_float(u3[i]);
+        }
+      }
+      if (j == n - 1) {
+        // Last tile of the row's range: causal diagonal, or the sequence's key bound.
+        const int lim = p.causal ? rpos : (len - 1);
+        const int cmax = lim - BN * j;
+#pragma unroll
+        for (int i = 0; i < 128; ++i)
+          if (i > cmax) s[i] = -INFINITY;
+      }
+      float mx = s[0];
+#pragma unroll
+      for (int i = 1; i < 128; ++i) mx = fmaxf(mx, s[i]);
+      const float mx2 = mx * c;
+      const bool need = mx2 > m_run + kRescaleThreshold;
+      const float m_new = need ? mx2 : m_run;
+      const float alpha = need ? ex2_approx(m_run - m_new) : 1.f;
+      if (j > 0 && __any_sync(0xffffffffu, need)) {
+        uint32_t u[32];
+#pragma unroll 1
+        for (int ch = 0; ch < D / 32; ++ch) {
+          tmem_ld32(tO + ch * 32, u);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * alpha);
+          tmem_st32(tO + ch * 32, u);
+        }
+      }
+      l_run *= alpha;
+      m_run = m_new;
+      const float mneg = (m_run == -INFINITY) ? 0.f : -m_run;
+      float sum = 0.f;
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float p0 = ex2_approx(fmaf(s[ch * 32 + 2 * i], c, mneg));
+          const float p1 = ex2_approx(fmaf(s[ch * 32 + 2 * i + 1], c, mneg));
+          sum += p0 + p1;
+          pk[i] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(tS + ch * 16, pk);
+      }
+      l_run += sum;
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[t]);
+    }
+    if (ok && n > 0) {
+      ok = __all_sync(0xffffffffu, mbar_wait(&o_final[t], 0, wc, kSiteOFinal));
+      if (ok) {
+        tc_fence_after();
+        const float inv = 1.f / l_run;
+        const bool valid = rpos < len;
+        __nv_bfloat16* orow = p.o + (size_t(start + rpos) * p.Hq + h) * D;
+#pragma unroll 1
+        for (int ch = 0; ch < D / 32; ++ch) {
+          uint32_t u[32];
+          tmem_ld32(tO + ch * 32, u);
+          tmem_wait_ld();
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            pk[i] = pack_bf16x2(__uint_as_float(u[2 * i]) * inv, __uint_as_float(u[2 * i + 1]) * inv);
+          if (valid) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+          }
+        }
+        if (valid) {
+          const float lse = (m_run + __log2f(l_run)) * 0.69314718055994530942f;
+          const size_t li = p.sv.cu ? size_t(h) * p.T + start + rpos
+                                    : (size_t(seq) * p.Hq + h) * p.sv.S + rpos;
+          p.lse[li] = lse;
+        }
+      }
+    }
+  }
+
+  // ---- teardown: every role has drained; release tensor memory.
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kWarpMMA) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+}  // namespace fwd
+}  // namespace attn_sm100

@@ -1,0 +1,335 @@
+// attn_lib.cu -- host side of libattn.so: argument validation, TMA descriptors,
+// launch configuration and the device status word.  The kernels live in the
+// included headers; this is the only translation unit of the library.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/attn.h"
+#include "attn_bwd.cuh"
+#include "attn_fwd.cuh"
+#include "umma_selftest.cuh"
+
+using namespace attn_sm100;
+
+// Sticky device status: [0] status bits, [1] site code of the first timeout.
+static __device__ unsigned g_attn_status[2];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::atomic<unsigned long long> g_timeout_ns{2000000000ull};
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+struct DeviceState {
+  bool ready = false;
+  bool sm100 = false;
+  unsigned* status = nullptr;
+};
+std::mutex g_mu;
+DeviceState g_dev[kMaxDevices];
+EncodeTiledFn g_encode = nullptr;
+
+// Per-device set-up (once): capability check, status-word address, kernel attributes.
+attn_status device_setup(DeviceState** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ATTN_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState& d = g_dev[dev];
+  if (!d.ready) {
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return ATTN_ERR_CUDA;
+    d.sm100 = (prop.major == 10 && prop.minor == 0);
+    if (d.sm100) {
+      if (!g_encode) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || !fn)
+          return ATTN_ERR_CUDA;
+        g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+      }
+      if (cudaGetSymbolAddress(reinterpret_cast<void**>(&d.status), g_attn_status) != cudaSuccess)
+        return ATTN_ERR_CUDA;
+      cudaError_t e = cudaSuccess;
+      e = e ? e : cudaFuncSetAttribute(fwd::attn_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, fwd::Cfg<64>::SMEM_ALLOC);
+      e = e ? e : cudaFuncSetAttribute(fwd::attn_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, fwd::Cfg<128>::SMEM_ALLOC);
+      e = e ? e : cudaFuncSetAttribute(bwd::attn_bwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, bwd::Cfg<64>::SMEM_ALLOC);
+      e = e ? e : cudaFuncSetAttribute(bwd::attn_bwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, bwd::Cfg<128>::SMEM_ALLOC);
+      e = e ? e : cudaFuncSetAttribute(selftest::umma_selftest_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, 32768 + 128 * 64 * 2 + 2048);
+      e = e ? e : cudaFuncSetAttribute(selftest::umma_selftest_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, 32768 + 128 * 128 * 2 + 2048);
+      if (e != cudaSuccess) return ATTN_ERR_CUDA;
+    }
+    d.ready = true;
+  }
+  if (!d.sm100) return ATTN_ERR_UNSUPPORTED;
+  *out = &d;
+  return ATTN_OK;
+}
+
+// 3-D view (D, H, T) of a [T][H][D] bf16 tensor; box 64 x 1 x 128, 128-byte swizzle.
+attn_status make_map(CUtensorMap* m, const void* base, int D, int H, long long T) {
+  const cuuint64_t dims[3] = {cuuint64_t(D), cuuint64_t(H), cuuint64_t(T)};
+  const cuuint64_t strides[2] = {cuuint64_t(D) * 2, cuuint64_t(H) * D * 2};
+  const cuuint32_t box[3] = {64, 1, 128};
+  const cuuint32_t es[3] = {1, 1, 1};
+  const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                              strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+attn_status check_sizes(int B, int Hq, int Hkv, int S, int D, float scale, bool varlen,
+                        long long* T) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || S < 1) return ATTN_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+  const long long t = varlen ? (long long)S : (long long)B * S;
+  // token coordinates are int32 in the kernels; keep every row index in range
+  if (t >= (1ll << 31) - 512 || ((t >> 7) + B + 1) * (long long)Hq >= (1ll << 31))
+    return ATTN_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+  *T = t;
+  return ATTN_OK;
+}
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+struct WsLayout {
+  size_t dq_acc, lse2, delta, total;
+  int ntile;
+};
+WsLayout ws_layout(int B, int Hq, long long T, int D) {
+  WsLayout w;
+  w.ntile = int((T >> 7) + B);
+  w.dq_acc = 0;
+  w.lse2 = round_up(size_t(T) * Hq * D * sizeof(float), 256);
+  w.delta = w.lse2 + round_up(size_t(Hq) * w.ntile * 128 * sizeof(float), 256);
+  w.total = w.delta + round_up(size_t(Hq) * w.ntile * 128 * sizeof(float), 256);
+  return w;
+}
+
+}  // namespace
+
+extern "C" {
+
+int attn_version(void) { return 100; }
+
+const char* attn_strerror(attn_status s) {
+  switch (s) {
+    case ATTN_OK: return "ok";
+    case ATTN_ERR_INVALID_ARG: return "invalid argument";
+    case ATTN_ERR_UNSUPPORTED: return "unsupported (head dim must be 64 or 128 on an sm_100 device)";
+    case ATTN_ERR_MISALIGNED: return "misaligned pointer";
+    case ATTN_ERR_CUDA: return "CUDA error";
+    case ATTN_ERR_TIMEOUT: return "device-side wait timed out";
+  }
+  return "unknown status";
+}
+
+void attn_set_wait_timeout_ns(unsigned long long ns) { g_timeout_ns.store(ns ? ns : 1); }
+
+attn_status attn_check_cu_seqlens(const int32_t* cu, int B, int S) {
+  if (!cu || B < 1 || S < 0) return ATTN_ERR_INVALID_ARG;
+  if (cu[0] != 0 || cu[B] != S) return ATTN_ERR_INVALID_ARG;
+  for (int b = 0; b < B; ++b)
+    if (cu[b + 1] < cu[b]) return ATTN_ERR_INVALID_ARG;
+  return ATTN_OK;
+}
+
+attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                     int Hq, int Hkv, int S, int D, int causal, float scale,
+                     const int32_t* cu_seqlens, void* stream) {
+  long long T = 0;
+  attn_status st = check_sizes(B, Hq, Hkv, S, D, scale, cu_seqlens != nullptr, &T);
+  if (st != ATTN_OK) return st;
+  if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+      !aligned(lse, 4) || (cu_seqlens && !aligned(cu_seqlens, 4)))
+    return ATTN_ERR_MISALIGNED;
+  DeviceState* dev = nullptr;
+  if ((st = device_setup(&dev)) != ATTN_OK) return st;
+
+  CUtensorMap mq, mk, mv;
+  if (make_map(&mq, q, D, Hq, T) || make_map(&mk, k, D, Hkv, T) || make_map(&mv, v, D, Hkv, T))
+    return ATTN_ERR_CUDA;
+  fwd::Params p;
+  p.sv = SeqView{cu_seqlens, B, cu_seqlens ? int(T) : S, int(T)};
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.Hq = Hq;
+  p.G = Hq / Hkv;
+  p.T = int(T);
+  p.causal = causal ? 1 : 0;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.nblk = int((T >> 8) + B);
+  p.status = dev->status;
+  p.timeout_ns = g_timeout_ns.load();
+  const dim3 grid(unsigned(p.nblk) * unsigned(Hq));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (D == 64)
+    fwd::attn_fwd_kernel<64><<<grid, fwd::kThreads, fwd::Cfg<64>::SMEM_ALLOC, s>>>(mq, mk, mv, p);
+  else
+    fwd::attn_fwd_kernel<128><<<grid, fwd::kThreads, fwd::Cfg<128>::SMEM_ALLOC, s>>>(mq, mk, mv, p);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+size_t attn_bwd_workspace_size(int B, int Hq, int S, int D, const int32_t* cu_seqlens) {
+  long long T = 0;
+  if (check_sizes(B, Hq, 1, S, D, 1.f, cu_seqlens != nullptr, &T) != ATTN_OK) return 0;
+  return ws_layout(B, Hq, T, D).total;
+}
+
+attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o,
+                     const float* lse, const void* dout, void* dq, void* dk, void* dv, int B,
+                     int Hq, int Hkv, int S, int D, int causal, float scale,
+                     const int32_t* cu_seqlens, void* workspace, size_t workspace_bytes,
+                     void* stream) {
+  long long T = 0;
+  attn_status st = check_sizes(B, Hq, Hkv, S, D, scale, cu_seqlens != nullptr, &T);
+  if (st != ATTN_OK) return st;
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !workspace)
+    return ATTN_ERR_INVALID_ARG;
+  const WsLayout w = ws_layout(B, Hq, T, D);
+  if (workspace_bytes < w.total) return ATTN_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+      !aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) ||
+      !aligned(lse, 4) || !aligned(workspace, 256) || (cu_seqlens && !aligned(cu_seqlens, 4)))
+    return ATTN_ERR_MISALIGNED;
+  DeviceState* dev = nullptr;
+  if ((st = device_setup(&dev)) != ATTN_OK) return st;
+
+  CUtensorMap mq, mk, mv, mdo;
+  if (make_map(&mq, q, D, Hq, T) || make_map(&mk, k, D, Hkv, T) || make_map(&mv, v, D, Hkv, T) ||
+      make_map(&mdo, dout, D, Hq, T))
+    return ATTN_ERR_CUDA;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* dq_acc = reinterpret_cast<float*>(ws + w.dq_acc);
+  float* lse2 = reinterpret_cast<float*>(ws + w.lse2);
+  float* delta = reinterpret_cast<float*>(ws + w.delta);
+  const SeqView sv{cu_seqlens, B, cu_seqlens ? int(T) : S, int(T)};
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  const dim3 pgrid(unsigned(w.ntile), unsigned(Hq));
+  if (D == 64)
+    bwd::bwd_preprocess_kernel<64><<<pgrid, 128, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, lse2,
+        delta, dq_acc, sv, Hq, int(T), w.ntile);
+  else
+    bwd::bwd_preprocess_kernel<128><<<pgrid, 128, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, lse2,
+        delta, dq_acc, sv, Hq, int(T), w.ntile);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+
+  bwd::Params p;
+  p.sv = sv;
+  p.dq_acc = dq_acc;
+  p.lse2 = lse2;
+  p.delta = delta;
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = Hq / Hkv;
+  p.T = int(T);
+  p.causal = causal ? 1 : 0;
+  p.ntile = w.ntile;
+  p.nkv = w.ntile;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.scale = scale;
+  p.status = dev->status;
+  p.timeout_ns = g_timeout_ns.load();
+  const dim3 grid(unsigned(p.nkv) * unsigned(Hkv));
+  if (D == 64)
+    bwd::attn_bwd_kernel<64><<<grid, bwd::kThreads, bwd::Cfg<64>::SMEM_ALLOC, s>>>(mq, mk, mv, mdo, p);
+  else
+    bwd::attn_bwd_kernel<128><<<grid, bwd::kThreads, bwd::Cfg<128>::SMEM_ALLOC, s>>>(mq, mk, mv, mdo, p);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+
+  const size_t n8 = size_t(T) * Hq * D / 8;
+  const unsigned cgrid = unsigned(n8 / 256 + 1 < 148 * 16 ? n8 / 256 + 1 : 148 * 16);
+  bwd::dq_convert_kernel<<<cgrid, 256, 0, s>>>(dq_acc, static_cast<__nv_bfloat16*>(dq), n8, scale);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+attn_status attn_device_status(void* stream, unsigned* site) {
+  DeviceState* dev = nullptr;
+  attn_status st = device_setup(&dev);
+  if (st != ATTN_OK) return st;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return ATTN_ERR_CUDA;
+  unsigned word[2] = {0, 0};
+  if (cudaMemcpy(word, dev->status, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  if (site) *site = word[1];
+  if (word[0] == 0) return ATTN_OK;
+  const unsigned zero[2] = {0, 0};
+  if (cudaMemcpy(dev->status, zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  return (word[0] & kStatusTimeout) ? ATTN_ERR_TIMEOUT : ATTN_ERR_CUDA;
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------------ self-tests
+static __global__ void wait_timeout_kernel(unsigned* status, unsigned long long timeout_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const WaitCtl wc{status, &abort_flag, timeout_ns};
+    mbar_wait(&bar, 0, wc, 0x400);  // nothing ever arrives: the wait gives up
+  }
+}
+
+extern "C" attn_status attn_selftest_wait_timeout(unsigned long long timeout_ns, void* stream) {
+  DeviceState* dev = nullptr;
+  attn_status st = device_setup(&dev);
+  if (st != ATTN_OK) return st;
+  if (timeout_ns == 0 || timeout_ns > 10000000000ull) return ATTN_ERR_INVALID_ARG;
+  wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(dev->status, timeout_ns);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+extern "C" attn_status attn_selftest_umma(int mode, int D, const void* a, const void* b,
+                                          const float* pin, const void* at, float* c,
+                                          void* stream) {
+  if (mode < 0 || mode > 2) return ATTN_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+  if (!b || !c || (mode == 0 && !a) || (mode == 1 && !pin) || (mode == 2 && !at))
+    return ATTN_ERR_INVALID_ARG;
+  if (!aligned(b, 16) || (a && !aligned(a, 16)) || (at && !aligned(at, 16)) ||
+      (pin && !aligned(pin, 16)) || !aligned(c, 16))
+    return ATTN_ERR_MISALIGNED;
+  DeviceState* dev = nullptr;
+  attn_status st = device_setup(&dev);
+  if (st != ATTN_OK) return st;
+  CUtensorMap ma, mb;
+  if (make_map(&ma, a ? a : b, D, 1, 128) || make_map(&mb, b, D, 1, 128)) return ATTN_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const unsigned long long to = g_timeout_ns.load();
+  if (D == 64)
+    selftest::umma_selftest_kernel<64><<<1, 128, 32768 + 128 * 64 * 2 + 2048, s>>>(
+        ma, mb, mode, pin, static_cast<const __nv_bfloat16*>(at), c, dev->status, to);
+  else
+    selftest::umma_selftest_kernel<128><<<1, 128, 32768 + 128 * 128 * 2 + 2048, s>>>(
+        ma, mb, mode, pin, static_cast<const __nv_bfloat16*>(at), c, dev->status, to);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}

@@ -1,0 +1,128 @@
+"""PyTorch-facing wrappers over the C ABI (torch supplies device memory and streams).
+
+    o, lse = attn_fwd(q, k, v, causal=True)                   # q [B,S,Hq,D], k/v [B,S,Hkv,D]
+    o, lse = attn_fwd(q, k, v, cu_seqlens=cu)                  # packed: q [T,Hq,D], cu int32 [n+1]
+    dq, dk, dv = attn_bwd(q, k, v, o, lse, do, causal=True)
+    o = attention(q, k, v, causal=True)                        # autograd-aware
+
+All arithmetic runs in libattn.so; these functions only check shapes, allocate
+outputs with torch and pass raw pointers and the current CUDA stream.
+"""
+from __future__ import annotations
+
+import math
+from typing import Optional, Tuple
+
+import torch
+
+from . import capi
+
+
+def _stream(device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _dims(q: torch.Tensor, k: torch.Tensor, cu_seqlens: Optional[torch.Tensor]):
+    if cu_seqlens is None:
+        if q.dim() != 4 or k.dim() != 4:
+            raise ValueError("dense inputs must be [B, S, H, D]")
+        B, S, Hq, D = q.shape
+        Hkv = k.shape[2]
+        if k.shape[0] != B or k.shape[1] != S or k.shape[3] != D:
+            raise ValueError("k/v shape does not match q")
+    else:
+        if q.dim() != 3 or k.dim() != 3:
+            raise ValueError("packed inputs must be [T, H, D]")
+        S, Hq, D = q.shape
+        Hkv = k.shape[1]
+        B = cu_seqlens.numel() - 1
+        if cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_cuda:
+            raise ValueError("cu_seqlens must be an int32 CUDA tensor")
+        if k.shape[0] != S or k.shape[2] != D:
+            raise ValueError("k/v shape does not match q")
+    return B, S, Hq, Hkv, D
+
+
+def _check_inputs(*ts: torch.Tensor) -> None:
+    for t in ts:
+        if not t.is_cuda:
+            raise ValueError("libattn needs CUDA tensors (there is no CPU path)")
+        if t.dtype != torch.bfloat16:
+            raise ValueError("tensors must be bfloat16")
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+
+
+def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = True,
+             scale: Optional[float] = None, cu_seqlens: Optional[torch.Tensor] = None,
+             out: Optional[torch.Tensor] = None,
+             lse: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Fused forward: returns (o, lse); lse is fp32 [B,Hq,S] (dense) or [Hq,T] (packed)."""
+    _check_inputs(q, k, v)
+    B, S, Hq, Hkv, D = _dims(q, k, cu_seqlens)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        shape = (Hq, S) if cu_seqlens is not None else (B, Hq, S)
+        lse = torch.empty(shape, dtype=torch.float32, device=q.device)
+    st = capi.attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                       B, Hq, Hkv, S, D, causal, scale,
+                       cu_seqlens.data_ptr() if cu_seqlens is not None else None,
+                       _stream(q.device))
+    capi.check(st, "attn_fwd")
+    return out, lse
+
+
+def attn_bwd_workspace_size(q: torch.Tensor, cu_seqlens: Optional[torch.Tensor] = None) -> int:
+    if cu_seqlens is None:
+        B, S, Hq, D = q.shape
+        return capi.attn_bwd_workspace_size(B, Hq, S, D, None)
+    S, Hq, D = q.shape
+    return capi.attn_bwd_workspace_size(cu_seqlens.numel() - 1, Hq, S, D, 1)
+
+
+def attn_bwd(q, k, v, o, lse, dout, causal: bool = True, scale: Optional[float] = None,
+             cu_seqlens: Optional[torch.Tensor] = None, dq=None, dk=None, dv=None,
+             workspace: Optional[torch.Tensor] = None):
+    """Fused backward: returns (dq, dk, dv)."""
+    _check_inputs(q, k, v, o, dout)
+    B, S, Hq, Hkv, D = _dims(q, k, cu_seqlens)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    need = attn_bwd_workspace_size(q, cu_seqlens)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    st = capi.attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                       dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                       B, Hq, Hkv, S, D, causal, scale,
+                       cu_seqlens.data_ptr() if cu_seqlens is not None else None,
+                       workspace.data_ptr(), workspace.numel(), _stream(q.device))
+    capi.check(st, "attn_bwd")
+    return dq, dk, dv
+
+
+class _FusedAttention(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, q, k, v, causal, scale, cu_seqlens):
+        o, lse = attn_fwd(q, k, v, causal=causal, scale=scale, cu_seqlens=cu_seqlens)
+        ctx.save_for_backward(q, k, v, o, lse, cu_seqlens)
+        ctx.causal, ctx.scale = causal, scale
+        return o
+
+    @staticmethod
+    def backward(ctx, do):
+        q, k, v, o, lse, cu = ctx.saved_tensors
+        dq, dk, dv = attn_bwd(q, k, v, o, lse, do.contiguous(), causal=ctx.causal,
+                              scale=ctx.scale, cu_seqlens=cu)
+        return dq, dk, dv, None, None, None
+
+
+def attention(q, k, v, causal: bool = True, scale: Optional[float] = None,
+              cu_seqlens: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Autograd-aware fused attention (forward and backward both in libattn.so)."""
+    return _FusedAttention.apply(q, k, v, causal, scale, cu_seqlens)

@@ -25,3 +25,17 @@ def pytest_collection_modifyitems(config, items):
     for it in items:
         if "gpu" in it.keywords:
             it.add_marker(skip)
+
+
+@pytest.fixture(autouse=True, scope="session")
+def _short_device_waits():
+    """GPU tests run with a 500 ms limit on every device-side wait (the library
+    default is 2 s), so that a broken pipeline gives up quickly."""
+    try:
+        import torch
+        if torch.cuda.is_available():
+            from long_context_attention_fwd_b200 import capi
+            capi.attn_set_wait_timeout_ns(500_000_000)
+    except Exception:
+        pass
+    yield

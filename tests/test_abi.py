@@ -1,0 +1,81 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports every
+function include/attn.h declares, and validates arguments before launching."""
+import ctypes
+
+import numpy as np
+import pytest
+
+from long_context_attention_fwd_b200 import capi
+
+
+def test_exports_every_declared_symbol():
+    lib = capi.lib()
+    names = capi.declared_symbols()
+    assert {"attn_fwd", "attn_bwd", "attn_bwd_workspace_size", "attn_strerror"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+        assert n in capi._SIGNATURES, n
+
+
+def test_version_and_strerror():
+    assert capi.attn_version() >= 100
+    for s in range(6):
+        assert capi.strerror(s)
+    assert capi.strerror(0) == "ok"
+
+
+A = 0x10000  # fake, 16-byte aligned addresses: validation fails before any CUDA call
+
+
+@pytest.mark.parametrize("args,want", [
+    ((0, 2, 2, 128, 64), capi.ATTN_ERR_INVALID_ARG),     # B = 0
+    ((1, 0, 2, 128, 64), capi.ATTN_ERR_INVALID_ARG),     # Hq = 0
+    ((1, 3, 2, 128, 64), capi.ATTN_ERR_INVALID_ARG),     # Hq % Hkv
+    ((1, 2, 2, 0, 64), capi.ATTN_ERR_INVALID_ARG),       # S = 0
+    ((1, 2, 2, 128, 96), capi.ATTN_ERR_UNSUPPORTED),     # D
+    ((1, 2, 2, 128, 256), capi.ATTN_ERR_UNSUPPORTED),
+])
+def test_fwd_validation(args, want):
+    B, Hq, Hkv, S, D = args
+    assert capi.attn_fwd(A, A, A, A, A, B, Hq, Hkv, S, D, 1, 0.125, None, None) == want
+
+
+def test_fwd_scale_and_pointers():
+    assert capi.attn_fwd(A, A, A, A, A, 1, 2, 2, 128, 64, 1, float("nan"), None, None) == 1
+    assert capi.attn_fwd(A, A, A, A, A, 1, 2, 2, 128, 64, 1, float("inf"), None, None) == 1
+    assert capi.attn_fwd(None, A, A, A, A, 1, 2, 2, 128, 64, 1, 0.1, None, None) == 1
+    assert capi.attn_fwd(A + 8, A, A, A, A, 1, 2, 2, 128, 64, 1, 0.1, None, None) == 3
+    assert capi.attn_fwd(A, A, A, A, A + 2, 1, 2, 2, 128, 64, 1, 0.1, None, None) == 3
+    assert capi.attn_fwd(A, A, A, A, A, 1, 2, 2, 128, 64, 1, 0.1, A + 2, None) == 3
+
+
+def test_bwd_validation_and_workspace():
+    ws = capi.attn_bwd_workspace_size(1, 28, 32768, 128, None)
+    T, Hq, D = 32768, 28, 128
+    ntile = T // 128 + 1
+    assert ws >= T * Hq * D * 4 + 2 * Hq * ntile * 128 * 4
+    assert capi.attn_bwd_workspace_size(0, 28, 32768, 128, None) == 0
+    assert capi.attn_bwd_workspace_size(1, 28, 32768, 96, None) == 0
+    # packed: S is the total token count, so the workspace does not scale with B
+    assert capi.attn_bwd_workspace_size(8, 28, 32768, 128, 1) < 1.01 * ws
+    args = [A] * 9 + [1, 2, 2, 128, 64, 1, 0.1, None]
+    need = capi.attn_bwd_workspace_size(1, 2, 128, 64, None)
+    assert capi.attn_bwd(*args, A, need - 1, None) == capi.ATTN_ERR_INVALID_ARG
+    assert capi.attn_bwd(*args, A + 16, need, None) == capi.ATTN_ERR_MISALIGNED
+    assert capi.attn_bwd(*args, None, need, None) == capi.ATTN_ERR_INVALID_ARG
+
+
+def test_check_cu_seqlens_host():
+    assert capi.attn_check_cu_seqlens([0, 3, 3, 10], 3, 10) == 0
+    assert capi.attn_check_cu_seqlens([0, 3, 2, 10], 3, 10) == 1
+    assert capi.attn_check_cu_seqlens([1, 3, 3, 10], 3, 10) == 1
+    assert capi.attn_check_cu_seqlens([0, 3, 3, 9], 3, 10) == 1
+    assert capi.attn_check_cu_seqlens([0, 3, 10], 3, 10) == 1
+
+
+def test_ops_refuses_cpu_tensors():
+    torch = pytest.importorskip("torch")
+    from long_context_attention_fwd_b200 import ops
+    q = torch.zeros(1, 128, 2, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        ops.attn_fwd(q, q, q)

@@ -1,0 +1,104 @@
+"""CUDA path vs the fp64 oracle on the same seeded bf16 inputs, through the C ABI.
+
+Small cases compare every element (several tiles, ragged tails, GQA, packed
+sequences with empty and one-token members, causal and full masks, both head
+dims).  The bar: O max |err| <= 1e-2, LSE max |err| <= 1e-3, dq/dk/dv relative
+L2 <= 1e-2, all against fp64 on the bf16-rounded inputs.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from helpers import (TOL_GRAD, TOL_LSE, GpuRun, make_case, o_error_report, oracle_args, rel_l2)
+from long_context_attention_fwd_b200 import inputs as I
+
+torch = pytest.importorskip("torch")
+
+SMALL = [
+    ("cfg0_tiny_S256_D64", I.workload(0)),
+    ("gqa4x2_S300_D128_causal", make_case(1, 4, 2, 300, 128, True, seed=11)),
+    ("gqa3x1_B2_S200_D64_causal", make_case(2, 3, 1, 200, 64, True, seed=12)),
+    ("mha2_S384_D128_full", make_case(1, 2, 2, 384, 128, False, seed=13)),
+    ("gqa2x1_S257_D64_full", make_case(1, 2, 1, 257, 64, False, seed=14)),
+    ("S1_D128", make_case(1, 2, 1, 1, 128, True, seed=15)),
+    ("S129_D64_unit", make_case(1, 2, 2, 129, 64, True, seed=16, qkv_mult=1.0)),
+    ("varlen_gqa4x2_D128_causal", make_case(0, 4, 2, 0, 128, True, seed=17,
+                                            lens=[5, 0, 300, 1, 129, 128, 700])),
+    ("varlen_mha2_D64_full", make_case(0, 2, 2, 0, 64, False, seed=18,
+                                       lens=[257, 3, 0, 130, 64])),
+    ("outliers_D64", make_case(1, 2, 2, 520, 64, True, seed=19, qkv_mult=1.0,
+                               outlier_p=0.01, outlier_mult=8.0)),
+    ("gqa7x1_S640_D128_causal", make_case(1, 7, 1, 640, 128, True, seed=20)),
+]
+
+
+def _ref(w, x):
+    q, k, v, do, kw = oracle_args(w, x)
+    o, lse = oracle.fwd(q, k, v, w.causal, w.softmax_scale, **kw)
+    dq, dk, dv = oracle.bwd(q, k, v, do, w.causal, w.softmax_scale, **kw)
+    return {"o": o, "lse": lse, "dq": dq, "dk": dk, "dv": dv}
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("name,w", SMALL, ids=[c[0] for c in SMALL])
+def test_small_elementwise(name, w):
+    run = GpuRun(w)
+    g = run.np_out()
+    r = _ref(w, run.x)
+    rep = o_error_report(g["o"], r["o"])
+    assert np.isfinite(g["o"]).all() and np.isfinite(g["lse"]).all()
+    assert rep["n_over"] == 0, rep
+    assert rep["max_abs"] <= 1e-2 or w.outlier_p > 0, rep
+    assert float(np.abs(g["lse"] - r["lse"]).max()) <= TOL_LSE
+    for name_ in ("dq", "dk", "dv"):
+        assert np.isfinite(g[name_]).all(), name_
+        e = rel_l2(g[name_], r[name_])
+        assert e <= TOL_GRAD, (name_, e)
+
+
+@pytest.mark.gpu
+def test_forward_and_dkdv_are_deterministic():
+    w = make_case(1, 4, 2, 700, 128, True, seed=21)
+    a = GpuRun(w)
+    b = GpuRun(w)
+    for t in ("o", "lse", "dk", "dv"):
+        assert torch.equal(getattr(a, t), getattr(b, t)), t
+    torch.testing.assert_close(a.dq.float(), b.dq.float(), rtol=0, atol=2e-2)
+
+
+@pytest.mark.gpu
+def test_packed_equals_separate_on_gpu():
+    lens = [300, 1, 0, 257, 128]
+    w = make_case(0, 4, 1, 0, 128, True, seed=22, lens=lens)
+    packed = GpuRun(w)
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    from long_context_attention_fwd_b200 import ops
+    for s, L in enumerate(lens):
+        if L == 0:
+            continue
+        a, b = int(cu[s]), int(cu[s + 1])
+        q = packed.q[a:b].unsqueeze(0).contiguous()
+        k = packed.k[a:b].unsqueeze(0).contiguous()
+        v = packed.v[a:b].unsqueeze(0).contiguous()
+        do = packed.do[a:b].unsqueeze(0).contiguous()
+        o, lse = ops.attn_fwd(q, k, v, causal=True, scale=w.softmax_scale)
+        dq, dk, dv = ops.attn_bwd(q, k, v, o, lse, do, causal=True, scale=w.softmax_scale)
+        assert torch.equal(o[0], packed.o[a:b])
+        assert torch.equal(lse[0], packed.lse[:, a:b])
+        assert torch.equal(dk[0], packed.dk[a:b])
+        assert torch.equal(dv[0], packed.dv[a:b])
+        torch.testing.assert_close(dq[0].float(), packed.dq[a:b].float(), rtol=0, atol=2e-2)
+
+
+@pytest.mark.gpu
+def test_autograd_wrapper_matches_explicit_calls():
+    from long_context_attention_fwd_b200 import ops
+    w = make_case(1, 2, 1, 256, 64, True, seed=23)
+    run = GpuRun(w)
+    q = run.q.clone().requires_grad_(True)
+    k = run.k.clone().requires_grad_(True)
+    v = run.v.clone().requires_grad_(True)
+    o = ops.attention(q, k, v, causal=True)
+    o.backward(run.do)
+    assert torch.equal(o.detach(), run.o)
+    assert torch.equal(k.grad, run.dk) and torch.equal(v.grad, run.dv)

@@ -1,0 +1,41 @@
+"""Failure detection on the GPU without a fault: a kernel waits on a barrier that
+nothing ever completes, its bounded wait gives up after the limit, the event is
+recorded in the status word, and the context stays usable afterwards."""
+import pytest
+
+from long_context_attention_fwd_b200 import capi
+
+torch = pytest.importorskip("torch")
+
+
+@pytest.mark.gpu
+def test_bounded_wait_reports_timeout_and_context_survives():
+    st, _ = capi.attn_device_status(None)  # clear anything left over
+    assert st in (capi.ATTN_OK, capi.ATTN_ERR_TIMEOUT)
+    capi.check(capi.attn_selftest_wait_timeout(2_000_000, None), "selftest")  # 2 ms limit
+    st, site = capi.attn_device_status(None)
+    assert st == capi.ATTN_ERR_TIMEOUT
+    assert site == 0x400
+    st, _ = capi.attn_device_status(None)
+    assert st == capi.ATTN_OK  # the record was cleared
+    # the context is still healthy: a real launch works and reports no error
+    from long_context_attention_fwd_b200 import ops
+    q = torch.randn(1, 128, 2, 64, device="cuda").bfloat16()
+    o, lse = ops.attn_fwd(q, q, q, causal=True)
+    torch.cuda.synchronize()
+    assert torch.isfinite(o.float()).all()
+    st, _ = capi.attn_device_status(None)
+    assert st == capi.ATTN_OK
+
+
+@pytest.mark.gpu
+def test_invalid_arguments_launch_nothing():
+    q = torch.zeros(1, 128, 3, 64, device="cuda", dtype=torch.bfloat16)
+    k = torch.zeros(1, 128, 2, 64, device="cuda", dtype=torch.bfloat16)
+    lse = torch.zeros(1, 3, 128, device="cuda")
+    st = capi.attn_fwd(q.data_ptr(), k.data_ptr(), k.data_ptr(), q.data_ptr(), lse.data_ptr(),
+                       1, 3, 2, 128, 64, 1, 0.125, None, None)
+    assert st == capi.ATTN_ERR_INVALID_ARG
+    st = capi.attn_fwd(q.data_ptr() + 2, k.data_ptr(), k.data_ptr(), q.data_ptr(), lse.data_ptr(),
+                       1, 2, 2, 128, 64, 1, 0.125, None, None)
+    assert st == capi.ATTN_ERR_MISALIGNED
