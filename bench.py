@@ -1,0 +1,379 @@
+#!/usr/bin/env python3
+"""Benchmark of the fused attention hot path (forward + backward) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+One step = attn_fwd + attn_bwd over one batch of the workload (default: the
+32K-token causal GQA case, Qwen2.5-7B attention shape: B=1, Hq=28, Hkv=4, D=128,
+S=32768), inputs resident in HBM.  Prints ONE JSON line on rank 0.
+
+FLOP convention: forward 4*S^2*D*Hq*B, halved when causal; backward 2.5x that.
+Under torchrun (N > 1) every rank runs its own independent batch (weak scaling,
+no collective on the data path); the reported time is the max over ranks.
+
+--impl reference times the fp64 CPU oracle (the reference arm of this build) on a
+bounded sample of the same workload: the first tokens of the causal sequence form
+an exact sub-problem, so each step runs the oracle's forward and backward on them.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from long_context_attention_fwd_b200 import inputs as I  # noqa: E402
+
+METRIC = "attn fwd/bwd TFLOP/s at S=32K causal GQA bf16; % of B200 BF16 peak"
+DEFAULT_WORKLOAD = "qwen2.5-7b_gqa28x4_S32768_D128"
+L2_BYTES = 126 * 2 ** 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured (MEASURED_PEAKS.json)"
+    return dict(FALLBACK_PEAKS), "fallback (no MEASURED_PEAKS.json)"
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def workload_config(w: I.Workload) -> dict:
+    cfg = {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "S": w.S, "D": w.D,
+           "causal": w.causal, "scale": w.softmax_scale,
+           "values": f"q,k,v ~ N(0,1)*{w.qkv_mult}, dO ~ N(0,1)*{w.do_mult}, seeded, bf16"}
+    if w.varlen is not None:
+        cfg["varlen_lengths"] = list(w.varlen)
+    return cfg
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_bench_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
+                stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[4:]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in rows:
+            for n, v in zip(names, r[3][1:]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        loaded = [r for r in rows if r[2] > 300.0] or rows
+        return {"sm_mhz": statistics.median(r[0] for r in loaded),
+                "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": sorted(reasons), "samples": len(rows),
+                "power_w_max": max(r[2] for r in rows)}
+
+
+# ---------------------------------------------------------------- CPU oracle
+def oracle_sample(w: I.Workload, tokens: int):
+    """The first `tokens` tokens of the workload's first sequence: an exact causal
+    sub-problem. Returns (callable running oracle fwd+bwd, FLOPs, description)."""
+    import oracle
+    sub = I.Workload(name=w.name + "_prefix", B=1, Hq=w.Hq, Hkv=w.Hkv, S=tokens, D=w.D,
+                     causal=w.causal, qkv_mult=w.qkv_mult, do_mult=w.do_mult, seed=w.seed)
+    x = I.make_inputs(sub)
+    q, k, v, do = (I.bf16_bits_to_f64(x[n]) for n in ("q", "k", "v", "do"))
+
+    def run():
+        oracle.fwd(q, k, v, sub.causal, sub.softmax_scale, B=1, S=tokens)
+        oracle.bwd(q, k, v, do, sub.causal, sub.softmax_scale, B=1, S=tokens)
+
+    flops = I.flop_fwd(sub) + I.flop_bwd(sub)
+    desc = (f"fp64 oracle fwd+bwd on a {tokens}-token causal prefix (exact sub-problem) "
+            f"with the workload's heads (Hq={w.Hq}, Hkv={w.Hkv}, D={w.D})")
+    return run, flops, desc
+
+
+def cpu_baseline(w: I.Workload, budget_s: float = 15.0):
+    import oracle
+    tokens = 1024 if w.D >= 128 else 2048
+    run, flops, desc = oracle_sample(w, tokens)
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        run()
+        n += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": flops * n / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+            "kind": "oracle", "sample": f"{desc}; {n} run(s) in {dt:.1f} s"}
+
+
+def run_reference(args, w: I.Workload):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    import oracle
+    tokens = 1024 if w.D >= 128 else 2048
+    run, flops, desc = oracle_sample(w, tokens)
+    for _ in range(args.warmup):
+        run()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        run()
+    dt = time.perf_counter() - t0
+    value = flops * args.steps / dt / 1e12
+    cores = oracle.num_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- GPU arm
+def run_gpu(args, w: I.Workload):
+    import torch
+    from long_context_attention_fwd_b200 import ops
+
+    ws, rank, local = dist_env()
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    dev = torch.device("cuda", local if ws > 1 else 0)
+    torch.cuda.set_device(dev)
+
+    # Each rank owns an independent batch: seed offset by rank.
+    wr = I.Workload(**{**w.__dict__, "seed": w.seed + 1000 * rank})
+    x = I.make_inputs(wr)
+    dense = wr.varlen is None
+    T = wr.tokens
+    shp_q = (wr.B, wr.S, wr.Hq, wr.D) if dense else (T, wr.Hq, wr.D)
+    shp_k = (wr.B, wr.S, wr.Hkv, wr.D) if dense else (T, wr.Hkv, wr.D)
+
+    def host_bf16(bits, shape):
+        t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16)
+        return t.view(shape).pin_memory()
+
+    hq, hk, hv, hdo = (host_bf16(x["q"], shp_q), host_bf16(x["k"], shp_k),
+                       host_bf16(x["v"], shp_k), host_bf16(x["do"], shp_q))
+    q, k, v, do = (t.to(dev) for t in (hq, hk, hv, hdo))
+    cu = None if dense else torch.from_numpy(x["cu_seqlens"]).to(dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((wr.Hq, T) if not dense else (wr.B, wr.Hq, wr.S), dtype=torch.float32,
+                      device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    wsp = torch.empty(ops.attn_bwd_workspace_size(q, cu), dtype=torch.uint8, device=dev)
+    scale = wr.softmax_scale
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        ops.attn_fwd(q, k, v, causal=wr.causal, scale=scale, cu_seqlens=cu, out=o, lse=lse)
+        if ev is not None:
+            ev[1].record(stream)
+        ops.attn_bwd(q, k, v, o, lse, do, causal=wr.causal, scale=scale, cu_seqlens=cu,
+                     dq=dq, dk=dk, dv=dv, workspace=wsp)
+        if ev is not None:
+            ev[2].record(stream)
+
+    def barrier():
+        if ws > 1:
+            import torch.distributed as dist
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    from long_context_attention_fwd_b200 import capi
+    st, site = capi.attn_device_status(stream.cuda_stream)
+    if st != 0:
+        raise RuntimeError(f"device status after warm-up: {capi.strerror(st)} site={site:#x}")
+
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    sampler.start()
+    time.sleep(0.3)
+    barrier()
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    t_end.record(stream)
+    barrier()
+    clocks = sampler.stop()
+    total_ms = t_start.elapsed_time(t_end)
+    fwd_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    bwd_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    st, site = capi.attn_device_status(stream.cuda_stream)
+    if st != 0:
+        raise RuntimeError(f"device status after timing: {capi.strerror(st)} site={site:#x}")
+
+    # end to end through the public API from pinned host buffers
+    ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    hdq = torch.empty(dq.shape, dtype=dq.dtype).pin_memory()
+    hdk = torch.empty(dk.shape, dtype=dk.dtype).pin_memory()
+    hdv = torch.empty(dv.shape, dtype=dv.dtype).pin_memory()
+    hlse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+
+    def e2e_step():
+        qd, kd, vd, dod = (t.to(dev, non_blocking=True) for t in (hq, hk, hv, hdo))
+        od, lsed = ops.attn_fwd(qd, kd, vd, causal=wr.causal, scale=scale, cu_seqlens=cu)
+        dqd, dkd, dvd = ops.attn_bwd(qd, kd, vd, od, lsed, dod, causal=wr.causal, scale=scale,
+                                     cu_seqlens=cu, workspace=wsp)
+        for h, d in ((ho, od), (hlse, lsed), (hdq, dqd), (hdk, dkd), (hdv, dvd)):
+            h.copy_(d, non_blocking=True)
+
+    e2e_steps = max(1, min(args.steps, 5))
+    e2e_step()
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    barrier()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdo))
+    d2h = sum(t.numel() * t.element_size() for t in (ho, hlse, hdq, hdk, hdv))
+
+    # max over ranks
+    if ws > 1:
+        import torch.distributed as dist
+        tt = torch.tensor([total_ms, e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms, e2e_ms = float(tt[0]), float(tt[1])
+
+    fl_f, fl_b = I.flop_fwd(wr), I.flop_bwd(wr)
+    ms_step = total_ms / args.steps
+    value = ws * (fl_f + fl_b) * args.steps / (total_ms * 1e-3) / 1e12
+    peaks, peaks_src = load_peaks()
+    peak_sus = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+    peak_burst = float(peaks.get("bf16_tflops"))
+    f_ms, b_ms = statistics.mean(fwd_ms), statistics.mean(bwd_ms)
+    fwd_tf = fl_f / (f_ms * 1e-3) / 1e12
+    bwd_tf = fl_b / (b_ms * 1e-3) / 1e12
+
+    traffic = None
+    tp = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tp):
+        try:
+            traffic = json.load(open(tp)).get(wr.name, {}).get("attn_bwd_kernel")
+        except Exception:
+            traffic = None
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": ws,
+            "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) inputs of the workload's shape)",
+            "config": {**workload_config(wr),
+                       "l2": f"no flush: q alone is {q.numel() * 2 / 2**20:.0f} MiB > 126 MiB L2",
+                       "parallelism": f"dp{ws} (independent batch per GPU)"},
+            "fwd_ms": f_ms, "bwd_ms": b_ms, "fwd_tflops": fwd_tf, "bwd_tflops": bwd_tf,
+            "fwd_frac_of_peak": fwd_tf / peak_sus, "bwd_frac_of_peak": bwd_tf / peak_sus,
+            "fwd_frac_of_burst_peak": fwd_tf / peak_burst,
+            "bwd_frac_of_burst_peak": bwd_tf / peak_burst,
+            "fwd_frac_of_nominal_2250": fwd_tf / 2250.0,
+            "bwd_frac_of_nominal_2250": bwd_tf / 2250.0,
+            "roofline": {
+                "bound": "tensor", "kernel": "attn_bwd (main kernel; time includes its two "
+                                             "small helper kernels, so frac is a lower bound)",
+                "achieved": bwd_tf, "peak": peak_sus, "unit": "TFLOP/s", "frac": bwd_tf / peak_sus,
+                "peak_source": f"{peaks_src}: bf16_tflops_sustained (kernel timed inside a "
+                               f"long step loop)",
+                "traffic": traffic,
+            },
+            "e2e": {"value": ws * (fl_f + fl_b) / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": e2e_ms},
+            "gpu_launches": 4 * args.steps,
+            "clocks": clocks,
+        }
+        if ws == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(wr)
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    w = I.workload(args.workload)
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_gpu(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

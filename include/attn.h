@@ -112,6 +112,11 @@ attn_status attn_selftest_wait_timeout(unsigned long long timeout_ns, void* stre
 attn_status attn_selftest_umma(int mode, int D, const void* a, const void* b, const float* p,
                                const void* at, float* c, void* stream);
 
+/* Description of the last failing CUDA call this library made on the calling thread
+ * ("" if none): the call's name and the CUDA error string.  Static per-thread
+ * storage, valid until the thread's next library call. */
+const char* attn_last_error(void);
+
 /* Library ABI version (major*100 + minor). */
 int attn_version(void);
 

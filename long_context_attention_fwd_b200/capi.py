@@ -26,7 +26,13 @@ ATTN_ERR_TIMEOUT = 5
 class AttnError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        super().__init__(f"{where}: {strerror(status)} (status {status})")
+        detail = ""
+        if status == ATTN_ERR_CUDA:
+            try:
+                detail = " [" + lib().attn_last_error().decode() + "]"
+            except Exception:
+                pass
+        super().__init__(f"{where}: {strerror(status)} (status {status}){detail}")
 
 
 _lock = threading.Lock()
@@ -49,6 +55,7 @@ _SIGNATURES = {
     "attn_selftest_wait_timeout": (_i, [ctypes.c_ulonglong, _vp]),
     "attn_selftest_umma": (_i, [_i, _i, _vp, _vp, _fp, _vp, _fp, _vp]),
     "attn_version": (_i, []),
+    "attn_last_error": (ctypes.c_char_p, []),
 }
 
 
@@ -137,3 +144,7 @@ def attn_selftest_umma(mode, D, a, b, p, at, c, stream=None) -> int:
 
 def attn_version() -> int:
     return lib().attn_version()
+
+
+def attn_last_error() -> str:
+    return lib().attn_last_error().decode()

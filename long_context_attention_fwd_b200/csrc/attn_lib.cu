@@ -7,6 +7,7 @@
 #include <atomic>
 #include <cmath>
 #include <cstdint>
+#include <cstdio>
 #include <cstring>
 #include <mutex>
 
@@ -21,6 +22,22 @@ using namespace attn_sm100;
 static __device__ unsigned g_attn_status[2];
 
 namespace {
+
+// Description of the last failing CUDA call made by this library on this thread.
+thread_local char g_last_error[256] = "";
+
+attn_status fail_cuda(const char* where, cudaError_t e) {
+  snprintf(g_last_error, sizeof(g_last_error), "%s: %s (%d)", where, cudaGetErrorString(e), int(e));
+  return ATTN_ERR_CUDA;
+}
+attn_status fail_cu(const char* where, CUresult r) {
+  snprintf(g_last_error, sizeof(g_last_error), "%s: CUresult %d", where, int(r));
+  return ATTN_ERR_CUDA;
+}
+attn_status check_launch(const char* where) {
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? ATTN_OK : fail_cuda(where, e);
+}
 
 constexpr int kMaxDevices = 64;
 std::atomic<unsigned long long> g_timeout_ns{2000000000ull};
@@ -42,25 +59,29 @@ EncodeTiledFn g_encode = nullptr;
 // Per-device set-up (once): capability check, status-word address, kernel attributes.
 attn_status device_setup(DeviceState** out) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ATTN_ERR_CUDA;
+  cudaError_t e0 = cudaGetDevice(&dev);
+  if (e0 != cudaSuccess) return fail_cuda("cudaGetDevice", e0);
+  if (dev < 0 || dev >= kMaxDevices) return fail_cuda("device index", cudaErrorInvalidDevice);
   std::lock_guard<std::mutex> lock(g_mu);
   DeviceState& d = g_dev[dev];
   if (!d.ready) {
     cudaDeviceProp prop;
-    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return ATTN_ERR_CUDA;
+    if ((e0 = cudaGetDeviceProperties(&prop, dev)) != cudaSuccess)
+      return fail_cuda("cudaGetDeviceProperties", e0);
     d.sm100 = (prop.major == 10 && prop.minor == 0);
     if (d.sm100) {
       if (!g_encode) {
         void* fn = nullptr;
         cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
-                cudaSuccess ||
-            q != cudaDriverEntryPointSuccess || !fn)
-          return ATTN_ERR_CUDA;
+        e0 = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+        if (e0 != cudaSuccess) return fail_cuda("cudaGetDriverEntryPoint", e0);
+        if (q != cudaDriverEntryPointSuccess || !fn)
+          return fail_cuda("cuTensorMapEncodeTiled lookup", cudaErrorSymbolNotFound);
         g_encode = reinterpret_cast<EncodeTiledFn>(fn);
       }
-      if (cudaGetSymbolAddress(reinterpret_cast<void**>(&d.status), g_attn_status) != cudaSuccess)
-        return ATTN_ERR_CUDA;
+      if ((e0 = cudaGetSymbolAddress(reinterpret_cast<void**>(&d.status), g_attn_status)) !=
+          cudaSuccess)
+        return fail_cuda("cudaGetSymbolAddress(status)", e0);
       cudaError_t e = cudaSuccess;
       e = e ? e : cudaFuncSetAttribute(fwd::attn_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, fwd::Cfg<64>::SMEM_ALLOC);
       e = e ? e : cudaFuncSetAttribute(fwd::attn_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, fwd::Cfg<128>::SMEM_ALLOC);
@@ -68,7 +89,7 @@ attn_status device_setup(DeviceState** out) {
       e = e ? e : cudaFuncSetAttribute(bwd::attn_bwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, bwd::Cfg<128>::SMEM_ALLOC);
       e = e ? e : cudaFuncSetAttribute(selftest::umma_selftest_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, 32768 + 128 * 64 * 2 + 2048);
       e = e ? e : cudaFuncSetAttribute(selftest::umma_selftest_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, 32768 + 128 * 128 * 2 + 2048);
-      if (e != cudaSuccess) return ATTN_ERR_CUDA;
+      if (e != cudaSuccess) return fail_cuda("cudaFuncSetAttribute", e);
     }
     d.ready = true;
   }
@@ -87,7 +108,7 @@ attn_status make_map(CUtensorMap* m, const void* base, int D, int H, long long T
                               strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
                               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
+  return r == CUDA_SUCCESS ? ATTN_OK : fail_cu("cuTensorMapEncodeTiled", r);
 }
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -128,6 +149,8 @@ extern "C" {
 
 int attn_version(void) { return 100; }
 
+const char* attn_last_error(void) { return g_last_error; }
+
 const char* attn_strerror(attn_status s) {
   switch (s) {
     case ATTN_OK: return "ok";
@@ -165,7 +188,7 @@ attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float
 
   CUtensorMap mq, mk, mv;
   if (make_map(&mq, q, D, Hq, T) || make_map(&mk, k, D, Hkv, T) || make_map(&mv, v, D, Hkv, T))
-    return ATTN_ERR_CUDA;
+    return ATTN_ERR_CUDA;  // reason recorded by make_map
   fwd::Params p;
   p.sv = SeqView{cu_seqlens, B, cu_seqlens ? int(T) : S, int(T)};
   p.o = static_cast<__nv_bfloat16*>(o);
@@ -184,7 +207,7 @@ attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float
     fwd::attn_fwd_kernel<64><<<grid, fwd::kThreads, fwd::Cfg<64>::SMEM_ALLOC, s>>>(mq, mk, mv, p);
   else
     fwd::attn_fwd_kernel<128><<<grid, fwd::kThreads, fwd::Cfg<128>::SMEM_ALLOC, s>>>(mq, mk, mv, p);
-  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  return check_launch("attn_fwd_kernel launch");
 }
 
 size_t attn_bwd_workspace_size(int B, int Hq, int S, int D, const int32_t* cu_seqlens) {
@@ -215,7 +238,7 @@ attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o,
   CUtensorMap mq, mk, mv, mdo;
   if (make_map(&mq, q, D, Hq, T) || make_map(&mk, k, D, Hkv, T) || make_map(&mv, v, D, Hkv, T) ||
       make_map(&mdo, dout, D, Hq, T))
-    return ATTN_ERR_CUDA;
+    return ATTN_ERR_CUDA;  // reason recorded by make_map
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   float* dq_acc = reinterpret_cast<float*>(ws + w.dq_acc);
   float* lse2 = reinterpret_cast<float*>(ws + w.lse2);
@@ -232,7 +255,7 @@ attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o,
     bwd::bwd_preprocess_kernel<128><<<pgrid, 128, 0, s>>>(
         static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, lse2,
         delta, dq_acc, sv, Hq, int(T), w.ntile);
-  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  if ((st = check_launch("bwd_preprocess_kernel launch")) != ATTN_OK) return st;
 
   bwd::Params p;
   p.sv = sv;
@@ -257,27 +280,28 @@ attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o,
     bwd::attn_bwd_kernel<64><<<grid, bwd::kThreads, bwd::Cfg<64>::SMEM_ALLOC, s>>>(mq, mk, mv, mdo, p);
   else
     bwd::attn_bwd_kernel<128><<<grid, bwd::kThreads, bwd::Cfg<128>::SMEM_ALLOC, s>>>(mq, mk, mv, mdo, p);
-  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  if ((st = check_launch("attn_bwd_kernel launch")) != ATTN_OK) return st;
 
   const size_t n8 = size_t(T) * Hq * D / 8;
   const unsigned cgrid = unsigned(n8 / 256 + 1 < 148 * 16 ? n8 / 256 + 1 : 148 * 16);
   bwd::dq_convert_kernel<<<cgrid, 256, 0, s>>>(dq_acc, static_cast<__nv_bfloat16*>(dq), n8, scale);
-  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  return check_launch("dq_convert_kernel launch");
 }
 
 attn_status attn_device_status(void* stream, unsigned* site) {
   DeviceState* dev = nullptr;
   attn_status st = device_setup(&dev);
   if (st != ATTN_OK) return st;
-  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return ATTN_ERR_CUDA;
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail_cuda("cudaStreamSynchronize", e);
   unsigned word[2] = {0, 0};
-  if (cudaMemcpy(word, dev->status, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess)
-    return ATTN_ERR_CUDA;
+  if ((e = cudaMemcpy(word, dev->status, sizeof(word), cudaMemcpyDeviceToHost)) != cudaSuccess)
+    return fail_cuda("cudaMemcpy(status)", e);
   if (site) *site = word[1];
   if (word[0] == 0) return ATTN_OK;
   const unsigned zero[2] = {0, 0};
-  if (cudaMemcpy(dev->status, zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
-    return ATTN_ERR_CUDA;
+  if ((e = cudaMemcpy(dev->status, zero, sizeof(zero), cudaMemcpyHostToDevice)) != cudaSuccess)
+    return fail_cuda("cudaMemcpy(status reset)", e);
   return (word[0] & kStatusTimeout) ? ATTN_ERR_TIMEOUT : ATTN_ERR_CUDA;
 }
 
@@ -305,7 +329,7 @@ extern "C" attn_status attn_selftest_wait_timeout(unsigned long long timeout_ns,
   if (st != ATTN_OK) return st;
   if (timeout_ns == 0 || timeout_ns > 10000000000ull) return ATTN_ERR_INVALID_ARG;
   wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(dev->status, timeout_ns);
-  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  return check_launch("wait_timeout_kernel launch");
 }
 
 extern "C" attn_status attn_selftest_umma(int mode, int D, const void* a, const void* b,
@@ -331,5 +355,5 @@ extern "C" attn_status attn_selftest_umma(int mode, int D, const void* a, const 
   else
     selftest::umma_selftest_kernel<128><<<1, 128, 32768 + 128 * 128 * 2 + 2048, s>>>(
         ma, mb, mode, pin, static_cast<const __nv_bfloat16*>(at), c, dev->status, to);
-  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  return check_launch("umma_selftest_kernel launch");
 }

@@ -27,6 +27,7 @@ multi-head case with outlier tails.
 from __future__ import annotations
 
 import math
+import os
 from dataclasses import dataclass, field
 from typing import List, Optional
 
@@ -69,26 +70,38 @@ def uniform(key: int, count: int, start: int = 0) -> np.ndarray:
     return (z >> np.uint64(11)).astype(np.float64) * (2.0 ** -53)
 
 
+def _normal_pairs(key: int, p0: int, p1: int) -> np.ndarray:
+    z = raw_u64(key, 2 * p0, 2 * (p1 - p0))
+    u1 = ((z[0::2] >> np.uint64(11)).astype(np.float64) + 1.0) * (2.0 ** -53)
+    u2 = (z[1::2] >> np.uint64(11)).astype(np.float64) * (2.0 ** -53)
+    r = np.sqrt(-2.0 * np.log(u1))
+    t = 2.0 * math.pi * u2
+    pair = np.empty(2 * (p1 - p0), dtype=np.float64)
+    pair[0::2] = r * np.cos(t)
+    pair[1::2] = r * np.sin(t)
+    return pair
+
+
 def normal(key: int, count: int) -> np.ndarray:
-    """``count`` standard normals (fp64), Box-Muller on pairs of draws."""
+    """``count`` standard normals (fp64), Box-Muller on pairs of draws.  Chunks are
+    independent (counter-based stream), so they are filled by a thread pool."""
     out = np.empty(count, dtype=np.float64)
     npairs = (count + 1) // 2
-    done = 0
-    p0 = 0
-    while p0 < npairs:
-        p1 = min(npairs, p0 + _CHUNK)
-        z = raw_u64(key, 2 * p0, 2 * (p1 - p0))
-        u1 = ((z[0::2] >> np.uint64(11)).astype(np.float64) + 1.0) * (2.0 ** -53)
-        u2 = (z[1::2] >> np.uint64(11)).astype(np.float64) * (2.0 ** -53)
-        r = np.sqrt(-2.0 * np.log(u1))
-        t = 2.0 * math.pi * u2
-        pair = np.empty(2 * (p1 - p0), dtype=np.float64)
-        pair[0::2] = r * np.cos(t)
-        pair[1::2] = r * np.sin(t)
-        n = min(count - done, pair.size)
-        out[done:done + n] = pair[:n]
-        done += n
-        p0 = p1
+    bounds = [(p0, min(npairs, p0 + _CHUNK)) for p0 in range(0, npairs, _CHUNK)]
+
+    def fill(b):
+        p0, p1 = b
+        pair = _normal_pairs(key, p0, p1)
+        n = min(count - 2 * p0, pair.size)
+        out[2 * p0:2 * p0 + n] = pair[:n]
+
+    if len(bounds) > 1:
+        from concurrent.futures import ThreadPoolExecutor
+        with ThreadPoolExecutor(max_workers=min(16, os.cpu_count() or 4)) as ex:
+            list(ex.map(fill, bounds))
+    else:
+        for b in bounds:
+            fill(b)
     return out
 
 

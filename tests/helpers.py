@@ -22,15 +22,23 @@ def bf16_ulp(x: np.ndarray) -> np.ndarray:
     return 2.0 ** (np.floor(np.log2(ax)) - 7)
 
 
-def o_error_report(o_gpu: np.ndarray, o_ref: np.ndarray) -> dict:
-    """Max |err| of a bf16 output against fp64, and the count of elements whose
-    error exceeds max(TOL_O, half a bf16 ulp of the reference) -- above |O| = 4
-    half an ulp is larger than TOL_O, so rounding alone can exceed it there."""
+def o_error_report(o_gpu: np.ndarray, o_ref: np.ndarray, o_absv: Optional[np.ndarray] = None) -> dict:
+    """Errors of a bf16 attention output against the fp64 oracle.
+
+    max_abs        max |O_gpu - O_ref| (the stated bar is 1e-2)
+    n_over_strict  elements above 1e-2
+    n_over_model   elements above max(1e-2, bound), bound = half a bf16 ulp of O_ref
+                   (output rounding) + 2^-8 * (P|V|)_i (P is rounded to bf16 before the
+                   PV product: relative error <= 2^-9 per probability, doubled for margin).
+                   o_absv = attention output with |V| in place of V, from the oracle.
+    """
     err = np.abs(o_gpu.astype(np.float64) - o_ref)
-    bound = np.maximum(TOL_O, 0.5 * bf16_ulp(o_ref) + 1e-3)
+    if o_absv is None:
+        o_absv = np.abs(o_ref)
+    bound = np.maximum(TOL_O, 0.5 * bf16_ulp(o_ref) + 2.0 ** -8 * np.abs(o_absv) + 1e-5)
     return {"max_abs": float(err.max()) if err.size else 0.0,
-            "n_over": int((err > bound).sum()),
-            "n_over_strict": int((err > TOL_O).sum())}
+            "n_over_strict": int((err > TOL_O).sum()),
+            "n_over_model": int((err > bound).sum())}
 
 
 def rel_l2(a: np.ndarray, b: np.ndarray) -> float:

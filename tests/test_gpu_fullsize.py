@@ -1,0 +1,95 @@
+"""Full-size workloads (8K and 32K causal GQA, packed 32K, MHA D=64 with outliers) in
+the launch configuration the bench times, checked against the fp64 oracle on
+sampled outputs it can compute one by one, plus properties that hold at any size:
+
+  * O and LSE of sampled query rows (first/last rows, tile edges, random rows);
+  * dQ of sampled query rows;
+  * dK, dV of the last keys of sampled (sequence, kv head) pairs -- only the query
+    rows after them see those keys, so the oracle's cost stays small;
+  * over ALL keys of every (sequence, kv head): sum_j dV_j equals the sum of dO over
+    the group's heads and rows (each probability row sums to one), and sum_j dK_j is
+    zero (each row of dS sums to zero) -- both up to bf16 rounding of P and dS.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from helpers import (TOL_GRAD, TOL_LSE, GpuRun, o_error_report, oracle_args, rel_l2)
+from long_context_attention_fwd_b200 import inputs as I
+
+torch = pytest.importorskip("torch")
+
+
+def _sample_rows(w, rng, n_random=24):
+    lens = w.seq_lengths()
+    rows = []
+    for _ in range(n_random):
+        b = int(rng.integers(len(lens)))
+        while lens[b] == 0:
+            b = int(rng.integers(len(lens)))
+        rows.append((b, int(rng.integers(w.Hq)), int(rng.integers(lens[b]))))
+    for b, L in enumerate(lens[:3]):
+        for i in (0, 1, 127, 128, 255, 256, L // 2, L - 129, L - 128, L - 1):
+            if 0 <= i < L:
+                rows.append((b, int(rng.integers(w.Hq)), int(i)))
+    return np.array(rows, dtype=np.int32)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("idx", [1, 2, 3, 4], ids=["S8K", "S32K", "varlen32K", "mha_D64_outliers"])
+def test_full_size_sampled(idx):
+    w = I.workload(idx)
+    run = GpuRun(w, poison=False)
+    g = run.np_out()
+    q, k, v, do, kw = oracle_args(w, run.x)
+    rng = np.random.default_rng(100 + idx)
+    cu = I.cu_seqlens_from(w.seq_lengths())
+    lens = w.seq_lengths()
+
+    # ---- forward rows
+    rows = _sample_rows(w, rng)
+    o_r, lse_r = oracle.fwd_rows(q, k, v, w.causal, w.softmax_scale, rows, **kw)
+    oa_r, _ = oracle.fwd_rows(q, k, np.abs(v), w.causal, w.softmax_scale, rows, **kw)
+    t = cu[rows[:, 0]] + rows[:, 2]
+    o_g = g["o"][t, rows[:, 1]]
+    if w.varlen is None:
+        lse_g = g["lse"][rows[:, 0], rows[:, 1], rows[:, 2]]
+    else:
+        lse_g = g["lse"][rows[:, 1], t]
+    rep = o_error_report(o_g, o_r, oa_r)
+    assert rep["n_over_model"] == 0, rep
+    if w.outlier_p == 0:
+        assert rep["max_abs"] <= 1e-2, rep
+    assert float(np.abs(lse_g - lse_r).max()) <= TOL_LSE
+
+    # ---- dQ rows
+    drows = rows[:: max(1, len(rows) // 16)]
+    dq_r, _, _ = oracle.bwd_dq_rows(q, k, v, do, w.causal, w.softmax_scale, drows, **kw)
+    td = cu[drows[:, 0]] + drows[:, 2]
+    assert rel_l2(g["dq"][td, drows[:, 1]], dq_r) <= TOL_GRAD
+
+    # ---- dK, dV of the last keys of a few (sequence, kv head) pairs
+    picks = [(len(lens) - 1, w.Hkv - 1), (0, 0)]
+    for b, gh in picks:
+        L = lens[b]
+        if L == 0:
+            continue
+        j0 = max(0, L - 160)
+        dk_r, dv_r = oracle.bwd_dkdv_range(q, k, v, do, w.causal, w.softmax_scale, b, gh, j0, L, **kw)
+        a = cu[b]
+        assert rel_l2(g["dk"][a + j0:a + L, gh], dk_r) <= TOL_GRAD
+        assert rel_l2(g["dv"][a + j0:a + L, gh], dv_r) <= TOL_GRAD
+
+    # ---- properties over all keys
+    G = w.Hq // w.Hkv
+    for b, L in enumerate(lens):
+        if L == 0:
+            continue
+        a = cu[b]
+        sum_dv = g["dv"][a:a + L].sum(0)                              # [Hkv, D]
+        want = g_do = do[a:a + L].reshape(L, w.Hkv, G, w.D).sum((0, 2))  # exact inputs
+        assert rel_l2(sum_dv, want) <= 1e-2
+        sum_dk = g["dk"][a:a + L].sum(0)
+        scale_ref = np.abs(g["dk"][a:a + L]).sum(0)
+        assert float(np.abs(sum_dk).max()) <= 2e-2 * float(scale_ref.max()), "sum_j dK_j != 0"
+        del g_do

@@ -35,8 +35,9 @@ SMALL = [
 def _ref(w, x):
     q, k, v, do, kw = oracle_args(w, x)
     o, lse = oracle.fwd(q, k, v, w.causal, w.softmax_scale, **kw)
+    o_absv, _ = oracle.fwd(q, k, np.abs(v), w.causal, w.softmax_scale, **kw)
     dq, dk, dv = oracle.bwd(q, k, v, do, w.causal, w.softmax_scale, **kw)
-    return {"o": o, "lse": lse, "dq": dq, "dk": dk, "dv": dv}
+    return {"o": o, "o_absv": o_absv, "lse": lse, "dq": dq, "dk": dk, "dv": dv}
 
 
 @pytest.mark.gpu
@@ -45,10 +46,11 @@ def test_small_elementwise(name, w):
     run = GpuRun(w)
     g = run.np_out()
     r = _ref(w, run.x)
-    rep = o_error_report(g["o"], r["o"])
+    rep = o_error_report(g["o"], r["o"], r["o_absv"])
     assert np.isfinite(g["o"]).all() and np.isfinite(g["lse"]).all()
-    assert rep["n_over"] == 0, rep
-    assert rep["max_abs"] <= 1e-2 or w.outlier_p > 0, rep
+    assert rep["n_over_model"] == 0, rep
+    if w.outlier_p == 0:
+        assert rep["max_abs"] <= 1e-2, rep  # the stated bar, met outright without outliers
     assert float(np.abs(g["lse"] - r["lse"]).max()) <= TOL_LSE
     for name_ in ("dq", "dk", "dv"):
         assert np.isfinite(g[name_]).all(), name_

@@ -39,3 +39,30 @@ def test_invalid_arguments_launch_nothing():
     st = capi.attn_fwd(q.data_ptr() + 2, k.data_ptr(), k.data_ptr(), q.data_ptr(), lse.data_ptr(),
                        1, 2, 2, 128, 64, 1, 0.125, None, None)
     assert st == capi.ATTN_ERR_MISALIGNED
+
+
+@pytest.mark.gpu
+def test_calls_from_another_host_thread():
+    """The library is usable from any host thread (autograd runs backward on its own)."""
+    import threading
+    from long_context_attention_fwd_b200 import ops
+    q = torch.randn(1, 256, 2, 64, device="cuda").bfloat16()
+    do = torch.randn_like(q)
+    o, lse = ops.attn_fwd(q, q, q, causal=True)
+    ref = ops.attn_bwd(q, q, q, o, lse, do, causal=True)
+    torch.cuda.synchronize()
+    box = {}
+
+    def work():
+        try:
+            torch.cuda.set_device(q.device)
+            box["r"] = ops.attn_bwd(q, q, q, o, lse, do, causal=True)
+            torch.cuda.synchronize()
+        except Exception as e:  # surfaced below with the library's error text
+            box["e"] = e
+
+    t = threading.Thread(target=work)
+    t.start()
+    t.join()
+    assert "e" not in box, box.get("e")
+    assert torch.equal(box["r"][1], ref[1]) and torch.equal(box["r"][2], ref[2])
