@@ -57,9 +57,22 @@ DeviceState g_dev[kMaxDevices];
 EncodeTiledFn g_encode = nullptr;
 
 // Per-device set-up (once): capability check, status-word address, kernel attributes.
-attn_status device_setup(DeviceState** out) {
+// `ptr` (optional) is a device pointer of the call: its device is made current on the
+// calling thread first, so that a call from any host thread (autograd's worker thread,
+// for one) runs on the device that owns the tensors with its context current.
+attn_status device_setup(DeviceState** out, const void* ptr = nullptr) {
   int dev = 0;
-  cudaError_t e0 = cudaGetDevice(&dev);
+  cudaError_t e0 = cudaSuccess;
+  if (ptr) {
+    cudaPointerAttributes attr;
+    e0 = cudaPointerGetAttributes(&attr, ptr);
+    if (e0 != cudaSuccess) return fail_cuda("cudaPointerGetAttributes", e0);
+    if (attr.type != cudaMemoryTypeDevice && attr.type != cudaMemoryTypeManaged)
+      return fail_cuda("tensor pointer is not device memory", cudaErrorInvalidValue);
+    e0 = cudaSetDevice(attr.device);
+    if (e0 != cudaSuccess) return fail_cuda("cudaSetDevice", e0);
+  }
+  e0 = cudaGetDevice(&dev);
   if (e0 != cudaSuccess) return fail_cuda("cudaGetDevice", e0);
   if (dev < 0 || dev >= kMaxDevices) return fail_cuda("device index", cudaErrorInvalidDevice);
   std::lock_guard<std::mutex> lock(g_mu);
@@ -184,7 +197,7 @@ attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float
       !aligned(lse, 4) || (cu_seqlens && !aligned(cu_seqlens, 4)))
     return ATTN_ERR_MISALIGNED;
   DeviceState* dev = nullptr;
-  if ((st = device_setup(&dev)) != ATTN_OK) return st;
+  if ((st = device_setup(&dev, q)) != ATTN_OK) return st;
 
   CUtensorMap mq, mk, mv;
   if (make_map(&mq, q, D, Hq, T) || make_map(&mk, k, D, Hkv, T) || make_map(&mv, v, D, Hkv, T))
@@ -233,7 +246,7 @@ attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o,
       !aligned(lse, 4) || !aligned(workspace, 256) || (cu_seqlens && !aligned(cu_seqlens, 4)))
     return ATTN_ERR_MISALIGNED;
   DeviceState* dev = nullptr;
-  if ((st = device_setup(&dev)) != ATTN_OK) return st;
+  if ((st = device_setup(&dev, q)) != ATTN_OK) return st;
 
   CUtensorMap mq, mk, mv, mdo;
   if (make_map(&mq, q, D, Hq, T) || make_map(&mk, k, D, Hkv, T) || make_map(&mv, v, D, Hkv, T) ||
@@ -343,7 +356,7 @@ extern "C" attn_status attn_selftest_umma(int mode, int D, const void* a, const 
       (pin && !aligned(pin, 16)) || !aligned(c, 16))
     return ATTN_ERR_MISALIGNED;
   DeviceState* dev = nullptr;
-  attn_status st = device_setup(&dev);
+  attn_status st = device_setup(&dev, b);
   if (st != ATTN_OK) return st;
   CUtensorMap ma, mb;
   if (make_map(&ma, a ? a : b, D, 1, 128) || make_map(&mb, b, D, 1, 128)) return ATTN_ERR_CUDA;
