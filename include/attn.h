@@ -62,8 +62,9 @@ attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float
                      const int32_t* cu_seqlens, void* stream);
 
 /* Bytes of device workspace attn_bwd needs for these arguments (same meaning as in
- * attn_bwd; only whether cu_seqlens is NULL matters).  Holds the fp32 dQ accumulator
- * [T][Hq][D], and Delta = rowsum(dO * O) and LSE*log2(e) in 128-row tiles.
+ * attn_bwd; only whether cu_seqlens is NULL matters).  Holds, per query head and
+ * 128-row query tile, the fp32 dQ accumulator tile, Delta = rowsum(dO * O) and
+ * LSE*log2(e); there are (T / 128) + B tiles per head (T = total tokens).
  * Returns 0 for invalid sizes. */
 size_t attn_bwd_workspace_size(int B, int Hq, int S, int D, const int32_t* cu_seqlens);
 

@@ -39,14 +39,13 @@ constexpr int kSlab = 128 * 128;
 
 struct Params {
   SeqView sv;
-  float* dq_acc;          // [T][Hq][D] fp32
+  float* dq_acc;          // [Hq][ntile][D/4][128][4] fp32: one contiguous block per query tile
   const float* lse2;      // [Hq][ntile][128]
   const float* delta;     // [Hq][ntile][128]
   __nv_bfloat16* dk;      // [T][Hkv][D]
   __nv_bfloat16* dv;
   int Hq, Hkv, G, T, causal;
-  int ntile;              // tiles per head in the lse2/delta workspace
-  int nkv;                // (T >> 7) + nseq: upper bound of 128-key blocks
+  int ntile;              // tiles per head in the workspace = (T >> 7) + nseq
   float scale_log2;
   float scale;
   unsigned* status;
@@ -56,6 +55,7 @@ struct Params {
 template <int D>
 struct Cfg {
   static constexpr int TILE = 128 * D * 2;  // one 128-row bf16 tile
+  static constexpr int DQ_TILE = 128 * D * 4;  // one 128-row fp32 dQ tile
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + TILE;
   static constexpr int OFF_Q = OFF_V + TILE;        // 2 stages
@@ -64,8 +64,9 @@ struct Cfg {
   static constexpr int OFF_LSE = OFF_DS + 128 * 128 * 2;  // 2 stages x 128 fp32
   static constexpr int OFF_DELTA = OFF_LSE + 2 * 512;
   static constexpr int OFF_BAR = OFF_DELTA + 2 * 512;
-  // kv_full, q_full[2], q_empty[2], s_full, dp_full, p_full, ds_full, dq_full, dq_free, dkv_final, drain
-  static constexpr int NBAR = 13;
+  // kv_full, q_full[2], q_empty[2], s_full, dp_full, p_full, ds_full, dq_full, dq_free,
+  // dkv_final, drain, stage_ready
+  static constexpr int NBAR = 14;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16;
   static constexpr int kMaxDyn = 232448;
@@ -74,15 +75,29 @@ struct Cfg {
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DQ = 128, COL_DV = 256, COL_DK = 256 + D;
   static_assert(SMEM_BYTES <= kMaxDyn, "shared memory budget");
+  // The fp32 dQ tile is staged in the Q and dO buffers of its own stage once the
+  // tile's MMAs are done: D=128 needs both (2 x 32 KB), D=64 the Q buffer alone.
+  static_assert(DQ_TILE <= 2 * TILE, "dQ staging must fit in one Q + dO stage");
 };
 
 enum : unsigned {
   kSiteKV = 0x200, kSiteQEmpty, kSiteQFull, kSiteSFull, kSiteDpFull, kSitePFull, kSiteDsFull,
-  kSiteDqFull, kSiteDqFree, kSiteFinal
+  kSiteDqFull, kSiteDqFree, kSiteFinal, kSiteStage
 };
 
+// dQ tile layout (workspace and staging): element (row r, column d) of a 128-row tile
+// lives at float offset ((d / 4) * 128 + r) * 4 + d % 4, so the 128 threads that each
+// own one row write 16-byte chunks to consecutive addresses (no bank conflicts) and
+// the whole tile is one contiguous block for a single bulk reduction.
+__host__ __device__ constexpr size_t dq_tile_offset(int r, int d) {
+  return (size_t(d >> 2) * 128 + r) * 4 + (d & 3);
+}
+
 // ---------------------------------------------------------------- preprocess
-// grid (nkv, Hq), 128 threads: one thread per query row of one 128-row tile.
+// grid (ntile, Hq), 128 threads: one thread per query row of one 128-row tile.
+// Writes Delta_i = dO_i . O_i and LSE_i * log2(e) into the tile-padded workspace
+// (+inf / 0 for rows past the sequence end, so their probabilities are exactly 0)
+// and zeroes the tile's fp32 dQ block.
 template <int D>
 __global__ void __launch_bounds__(128)
 bwd_preprocess_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
@@ -116,29 +131,38 @@ bwd_preprocess_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* 
     dl = acc;
     const size_t li = sv.cu ? size_t(h) * T + start + qpos : (size_t(seq) * Hq + h) * sv.S + qpos;
     l2 = lse[li] * 1.4426950408889634f;
-    float4* z = reinterpret_cast<float4*>(dq_acc + row);
-#pragma unroll 4
-    for (int i = 0; i < D / 4; ++i) z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
   const size_t wi = (size_t(h) * ntile + blockIdx.x) * 128 + r;
   lse2[wi] = l2;
   delta[wi] = dl;
+  float4* z = reinterpret_cast<float4*>(dq_acc + (size_t(h) * ntile + blockIdx.x) * 128 * D);
+#pragma unroll 4
+  for (int i = 0; i < D / 4; ++i) z[i * 128 + r] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
 // ---------------------------------------------------------------- dq convert
+// grid (ntile, Hq), 256 threads: dq[t][h][:] = bf16(scale * dQ tile rows), 8 columns per item.
+template <int D>
 __global__ void __launch_bounds__(256)
-dq_convert_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ dq, size_t n8,
-                  float scale) {
-  for (size_t i = blockIdx.x * size_t(blockDim.x) + threadIdx.x; i < n8;
-       i += size_t(gridDim.x) * blockDim.x) {
-    const float4 a = __ldg(reinterpret_cast<const float4*>(acc) + 2 * i);
-    const float4 b = __ldg(reinterpret_cast<const float4*>(acc) + 2 * i + 1);
+dq_convert_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ dq, SeqView sv,
+                  int Hq, int ntile, float scale) {
+  int seq, m, start, len;
+  if (!locate_block<7>(sv, blockIdx.x, seq, m, start, len)) return;
+  const int h = blockIdx.y;
+  const float4* blk = reinterpret_cast<const float4*>(acc + (size_t(h) * ntile + blockIdx.x) * 128 * D);
+  constexpr int G8 = D / 8;
+  for (int idx = threadIdx.x; idx < 128 * G8; idx += 256) {
+    const int r = idx / G8, c8 = idx % G8;
+    const int qpos = m * 128 + r;
+    if (qpos >= len) continue;
+    const float4 a = __ldg(blk + (2 * c8) * 128 + r);
+    const float4 b = __ldg(blk + (2 * c8 + 1) * 128 + r);
     uint4 out;
     out.x = pack_bf16x2(a.x * scale, a.y * scale);
     out.y = pack_bf16x2(a.z * scale, a.w * scale);
     out.z = pack_bf16x2(b.x * scale, b.y * scale);
     out.w = pack_bf16x2(b.z * scale, b.w * scale);
-    reinterpret_cast<uint4*>(dq)[i] = out;
+    *reinterpret_cast<uint4*>(dq + (size_t(start + qpos) * Hq + h) * D + 8 * c8) = out;
   }
 }
 
@@ -181,6 +205,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   uint64_t* dq_free = bars + 10;
   uint64_t* dkv_final = bars + 11;
   uint64_t* drain = bars + 12;
+  uint64_t* stage_ready = bars + 13;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   float* lse_s = reinterpret_cast<float*>(smem + C::OFF_LSE);
@@ -201,6 +226,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     mbar_init(dq_free, 4);
     mbar_init(dkv_final, 1);
     mbar_init(drain, 1);
+    mbar_init(stage_ready, 4);
     fence_mbar_init();
   }
   if (warp == kWarpMMA) {
@@ -304,8 +330,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         for (int kk = 0; kk < 8; ++kk)  // dQ_tile = dS K
           mma_ss(tmem + C::COL_DQ, sdesc_sw128(dsb + kk * 2048, 16384, 1024),
                  sdesc_sw128(kb + kk * 2048, kSlab, 1024), idQ, kk > 0 ? 1u : 0u);
-        mma_commit(dq_full);
-        mma_commit(&q_empty[st]);
+        mma_commit(dq_full);  // the stage is released by the dQ warps after staging
       }
       if (ok) mma_commit(dkv_final);
       mma_commit(drain);
@@ -348,10 +373,17 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
       }
       const bool diag = p.causal && m == n;
+      const float4* lse4 = reinterpret_cast<const float4*>(lse_t);
 #pragma unroll
-      for (int i = 0; i < 128; ++i) {
-        const float e = ex2_approx(fmaf(pr[i], c, -lse_t[i]));
-        pr[i] = (key_ok && !(diag && i < r)) ? e : 0.f;
+      for (int i4 = 0; i4 < 32; ++i4) {
+        const float4 l4 = lse4[i4];
+        const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int i = 4 * i4 + u;
+          const float e = ex2_approx(fmaf(pr[i], c, -lv[u]));
+          pr[i] = (key_ok && !(diag && i < r)) ? e : 0.f;
+        }
       }
 #pragma unroll
       for (int ch = 0; ch < 4; ++ch) {
@@ -377,12 +409,15 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tmem_ld32(tP + ch * 32, u);
         tmem_wait_ld();
         uint32_t pk[16];
+        const float4* dl4 = reinterpret_cast<const float4*>(dlt_t + ch * 32);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int c0 = ch * 32 + 2 * i;
-          const float d0 = pr[c0] * (__uint_as_float(u[2 * i]) - dlt_t[c0]);
-          const float d1 = pr[c0 + 1] * (__uint_as_float(u[2 * i + 1]) - dlt_t[c0 + 1]);
-          pk[i] = pack_bf16x2(d0, d1);
+        for (int i4 = 0; i4 < 8; ++i4) {
+          const float4 d4 = dl4[i4];
+          const int c0 = ch * 32 + 4 * i4;
+          pk[2 * i4] = pack_bf16x2(pr[c0] * (__uint_as_float(u[4 * i4]) - d4.x),
+                                   pr[c0 + 1] * (__uint_as_float(u[4 * i4 + 1]) - d4.y));
+          pk[2 * i4 + 1] = pack_bf16x2(pr[c0 + 2] * (__uint_as_float(u[4 * i4 + 2]) - d4.z),
+                                       pr[c0 + 3] * (__uint_as_float(u[4 * i4 + 3]) - d4.w));
         }
         tmem_st16(tP + ch * 16, pk);
         // shared memory: query rows ch*32 .. ch*32+31 -> 64-row block ch/2, 16-byte chunks
@@ -427,36 +462,61 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
   } else {
     // ------------------------------------------------------------ dQ drain (warps 4-7)
+    // Per query tile: read dQ_tile from TMEM (thread = row), free the TMEM columns,
+    // write the rows into this stage's Q/dO buffers (the tile's MMAs are done with
+    // them) in the workspace's tile layout, then one thread issues a bulk fp32
+    // reduce-add of the whole tile into the workspace and releases the stage.
     const int qw = warp & 3;
     const int r = qw * 32 + lane;      // query row of the tile (dQ) / key row (dK epilogue)
     const uint32_t tQ = tmem_addr(tmem, qw * 32, C::COL_DQ);
     bool ok = true;
     for (int it = 0; it < iters; ++it) {
+      const int st = it & 1;
       const int hq = g * p.G + it / per_head;
       const int m = m0 + it % per_head;
       ok = __all_sync(0xffffffffu, mbar_wait(dq_full, it & 1, wc, kSiteDqFull));
       if (!ok) break;
       tc_fence_after();
-      float acc[D];
+      uint32_t acc[D];
 #pragma unroll
       for (int ch = 0; ch < D / 32; ++ch) {
         uint32_t u[32];
         tmem_ld32(tQ + ch * 32, u);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) acc[ch * 32 + i] = __uint_as_float(u[i]);
+        for (int i = 0; i < 32; ++i) acc[ch * 32 + i] = u[i];
       }
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(dq_free);
-      const int qpos = m * 128 + r;
-      if (qpos < len) {
-        float4* dst = reinterpret_cast<float4*>(p.dq_acc + (size_t(start + qpos) * p.Hq + hq) * D);
+      uint8_t* stage_q = smem + C::OFF_Q + st * C::TILE;
+      uint8_t* stage_do = smem + C::OFF_DO + st * C::TILE;
 #pragma unroll
-        for (int i = 0; i < D / 4; ++i)
-          atomicAdd(dst + i, make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]));
+      for (int c4 = 0; c4 < D / 4; ++c4) {
+        uint8_t* dst = (c4 * 2048 < C::TILE) ? stage_q + c4 * 2048 : stage_do + (c4 * 2048 - C::TILE);
+        *reinterpret_cast<uint4*>(dst + r * 16) =
+            make_uint4(acc[4 * c4], acc[4 * c4 + 1], acc[4 * c4 + 2], acc[4 * c4 + 3]);
       }
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(stage_ready);
+      if (qw == 0 && lane == 0) {
+        if (mbar_wait(stage_ready, it & 1, wc, kSiteStage)) {
+          float* dst = p.dq_acc + (size_t(hq) * p.ntile + tile_base + m) * 128 * D;
+          if (C::DQ_TILE > C::TILE) {
+            bulk_reduce_add_f32(dst, stage_q, C::TILE);
+            bulk_reduce_add_f32(dst + C::TILE / 4, stage_do, C::DQ_TILE - C::TILE);
+          } else {
+            bulk_reduce_add_f32(dst, stage_q, C::DQ_TILE);
+          }
+          bulk_commit();
+          bulk_wait_read0();
+          mbar_arrive(&q_empty[st]);
+        }
+      }
+      __syncwarp();
     }
+    if (qw == 0 && lane == 0) bulk_wait0();
     // epilogue: dK rows (scaled)
     if (ok) {
       ok = __all_sync(0xffffffffu, mbar_wait(dkv_final, 0, wc, kSiteFinal));

@@ -266,7 +266,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const uint32_t tS = tmem_addr(tmem, qw * 32, colS);
     const uint32_t tO = tmem_addr(tmem, qw * 32, colO);
     float m_run = -INFINITY;  // reference maximum (log2 units) the accumulator is scaled to
-    float l_run = 0.f;        // running normaliser relative to m_run
+    float l_run = 0.f;        // running normaliser relative to m_run (fp32 probabilities)
+    float lb_run = 0.f;       // the same over the bf16-rounded probabilities fed to PV
     bool ok = true;
     for (int j = 0; j < n; ++j) {
       ok = __all_sync(0xffffffffu, mbar_wait(&s_full[t], j & 1, wc, kSiteSFull));
@@ -296,9 +297,20 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         for (int i = 0; i < 128; ++i)
           if (i > cmax) s[i] = -INFINITY;
       }
-      float mx = s[0];
+      float mx;
+      {
+        float m4[4] = {s[0], s[1], s[2], s[3]};
 #pragma unroll
-      for (int i = 1; i < 128; ++i) mx = fmaxf(mx, s[i]);
+        for (int i = 4; i < 124; i += 8) {  // elements 4 .. 123
+          m4[0] = fmax3(m4[0], s[i], s[i + 4]);
+          m4[1] = fmax3(m4[1], s[i + 1], s[i + 5]);
+          m4[2] = fmax3(m4[2], s[i + 2], s[i + 6]);
+          m4[3] = fmax3(m4[3], s[i + 3], s[i + 7]);
+        }
+        m4[0] = fmax3(m4[0], s[124], s[125]);
+        m4[1] = fmax3(m4[1], s[126], s[127]);
+        mx = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]);
+      }
       const float mx2 = mx * c;
       const bool need = mx2 > m_run + kRescaleThreshold;
       const float m_new = need ? mx2 : m_run;
@@ -315,22 +327,36 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
       }
       l_run *= alpha;
+      lb_run *= alpha;
       m_run = m_new;
       const float mneg = (m_run == -INFINITY) ? 0.f : -m_run;
-      float sum = 0.f;
+      const uint64_t cc = f2_pack(c, c), mm = f2_pack(mneg, mneg);
+      // Two running sums: of the fp32 probabilities (for the log-sum-exp) and of
+      // their bf16 roundings (the values the PV MMA consumes), so that O is
+      // normalised by exactly the weights it was accumulated with.
+      uint64_t sf[4] = {0, 0, 0, 0}, sb[4] = {0, 0, 0, 0};
 #pragma unroll
       for (int ch = 0; ch < 4; ++ch) {
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float p0 = ex2_approx(fmaf(s[ch * 32 + 2 * i], c, mneg));
-          const float p1 = ex2_approx(fmaf(s[ch * 32 + 2 * i + 1], c, mneg));
-          sum += p0 + p1;
-          pk[i] = pack_bf16x2(p0, p1);
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(s[ch * 32 + 2 * i], s[ch * 32 + 2 * i + 1]), cc, mm), x0, x1);
+          const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+          const uint32_t b = pack_bf16x2(p0, p1);
+          pk[i] = b;
+          sf[i & 3] = f2_add(sf[i & 3], f2_pack(p0, p1));
+          sb[i & 3] = f2_add(sb[i & 3], f2_pack(__uint_as_float(b << 16), __uint_as_float(b & 0xFFFF0000u)));
         }
         tmem_st16(tS + ch * 16, pk);
       }
-      l_run += sum;
+      {
+        float a0, a1, b0, b1;
+        f2_unpack(f2_add(f2_add(sf[0], sf[1]), f2_add(sf[2], sf[3])), a0, a1);
+        f2_unpack(f2_add(f2_add(sb[0], sb[1]), f2_add(sb[2], sb[3])), b0, b1);
+        l_run += a0 + a1;
+        lb_run += b0 + b1;
+      }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -340,7 +366,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       ok = __all_sync(0xffffffffu, mbar_wait(&o_final[t], 0, wc, kSiteOFinal));
       if (ok) {
         tc_fence_after();
-        const float inv = 1.f / l_run;
+        const float inv = 1.f / lb_run;
         const bool valid = rpos < len;
         __nv_bfloat16* orow = p.o + (size_t(start + rpos) * p.Hq + h) * D;
 #pragma unroll 1

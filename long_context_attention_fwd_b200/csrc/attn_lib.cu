@@ -150,7 +150,7 @@ WsLayout ws_layout(int B, int Hq, long long T, int D) {
   WsLayout w;
   w.ntile = int((T >> 7) + B);
   w.dq_acc = 0;
-  w.lse2 = round_up(size_t(T) * Hq * D * sizeof(float), 256);
+  w.lse2 = round_up(size_t(Hq) * w.ntile * 128 * D * sizeof(float), 256);
   w.delta = w.lse2 + round_up(size_t(Hq) * w.ntile * 128 * sizeof(float), 256);
   w.total = w.delta + round_up(size_t(Hq) * w.ntile * 128 * sizeof(float), 256);
   return w;
@@ -283,21 +283,23 @@ attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o,
   p.T = int(T);
   p.causal = causal ? 1 : 0;
   p.ntile = w.ntile;
-  p.nkv = w.ntile;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.scale = scale;
   p.status = dev->status;
   p.timeout_ns = g_timeout_ns.load();
-  const dim3 grid(unsigned(p.nkv) * unsigned(Hkv));
+  const dim3 grid(unsigned(w.ntile) * unsigned(Hkv));
   if (D == 64)
     bwd::attn_bwd_kernel<64><<<grid, bwd::kThreads, bwd::Cfg<64>::SMEM_ALLOC, s>>>(mq, mk, mv, mdo, p);
   else
     bwd::attn_bwd_kernel<128><<<grid, bwd::kThreads, bwd::Cfg<128>::SMEM_ALLOC, s>>>(mq, mk, mv, mdo, p);
   if ((st = check_launch("attn_bwd_kernel launch")) != ATTN_OK) return st;
 
-  const size_t n8 = size_t(T) * Hq * D / 8;
-  const unsigned cgrid = unsigned(n8 / 256 + 1 < 148 * 16 ? n8 / 256 + 1 : 148 * 16);
-  bwd::dq_convert_kernel<<<cgrid, 256, 0, s>>>(dq_acc, static_cast<__nv_bfloat16*>(dq), n8, scale);
+  if (D == 64)
+    bwd::dq_convert_kernel<64><<<pgrid, 256, 0, s>>>(dq_acc, static_cast<__nv_bfloat16*>(dq), sv, Hq,
+                                                    w.ntile, scale);
+  else
+    bwd::dq_convert_kernel<128><<<pgrid, 256, 0, s>>>(dq_acc, static_cast<__nv_bfloat16*>(dq), sv,
+                                                     Hq, w.ntile, scale);
   return check_launch("dq_convert_kernel launch");
 }
 

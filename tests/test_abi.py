@@ -57,7 +57,8 @@ def test_bwd_validation_and_workspace():
     assert capi.attn_bwd_workspace_size(0, 28, 32768, 128, None) == 0
     assert capi.attn_bwd_workspace_size(1, 28, 32768, 96, None) == 0
     # packed: S is the total token count, so the workspace does not scale with B
-    assert capi.attn_bwd_workspace_size(8, 28, 32768, 128, 1) < 1.01 * ws
+    # (only one padding tile per sequence and head is added)
+    assert capi.attn_bwd_workspace_size(8, 28, 32768, 128, 1) < 1.05 * ws
     args = [A] * 9 + [1, 2, 2, 128, 64, 1, 0.1, None]
     need = capi.attn_bwd_workspace_size(1, 2, 128, 64, None)
     assert capi.attn_bwd(*args, A, need - 1, None) == capi.ATTN_ERR_INVALID_ARG
