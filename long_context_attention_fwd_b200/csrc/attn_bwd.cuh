@@ -23,7 +23,8 @@
 //   dq_convert      dq = bf16(scale * accumulator).
 //
 // Warps: 0-3 compute P^T and dS^T (one thread per key row), 4-7 drain dQ from TMEM
-// into the accumulator, 8 is the TMA producer, 9 issues the MMAs.
+// and bulk-reduce it into the accumulator, 8 is the TMA producer, 9 issues the MMAs,
+// 10-11 only complete the control warpgroup for the register split.
 #pragma once
 #include <cuda_bf16.h>
 #include "attn_common.cuh"
@@ -32,9 +33,16 @@
 namespace attn_sm100 {
 namespace bwd {
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;    // 12 warps; warps 10-11 only complete the control warpgroup
 constexpr int kWarpTMA = 8;
 constexpr int kWarpMMA = 9;
+// Register split (setmaxnreg): the launch gives every thread 168 registers
+// (384 x 168 = 64512); the control warpgroup (warps 8-11) drops to 72 and the two
+// compute warpgroups rise to 216: 128 x 72 + 256 x 216 = 64512, exactly the pool.
+constexpr int kRegsLaunch = 168;
+constexpr int kRegsControl = 72;
+constexpr int kRegsCompute = 216;
+static_assert(128 * kRegsControl + 256 * kRegsCompute <= kThreads * kRegsLaunch, "register split");
 constexpr int kSlab = 128 * 128;
 
 struct Params {
@@ -64,9 +72,9 @@ struct Cfg {
   static constexpr int OFF_LSE = OFF_DS + 128 * 128 * 2;  // 2 stages x 128 fp32
   static constexpr int OFF_DELTA = OFF_LSE + 2 * 512;
   static constexpr int OFF_BAR = OFF_DELTA + 2 * 512;
-  // kv_full, q_full[2], q_empty[2], s_full, dp_full, p_full, ds_full, dq_full, dq_free,
-  // dkv_final, drain, stage_ready
-  static constexpr int NBAR = 14;
+  // kv_full, q_full[2], q_empty[2], do_full[2], do_empty[2], s_full, dp_full, p_full, ds_full,
+  // dq_full, dq_free, ds_free, stage_a, stage_b, dkv_final, drain
+  static constexpr int NBAR = 20;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16;
   static constexpr int kMaxDyn = 232448;
@@ -75,14 +83,14 @@ struct Cfg {
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DQ = 128, COL_DV = 256, COL_DK = 256 + D;
   static_assert(SMEM_BYTES <= kMaxDyn, "shared memory budget");
-  // The fp32 dQ tile is staged in the Q and dO buffers of its own stage once the
-  // tile's MMAs are done: D=128 needs both (2 x 32 KB), D=64 the Q buffer alone.
-  static_assert(DQ_TILE <= 2 * TILE, "dQ staging must fit in one Q + dO stage");
+  // The fp32 dQ tile is staged in the dS buffer (32 KB) and, for D = 128, in the dO
+  // buffer of its own stage (32 KB) once the tile's MMAs are done with them.
+  static_assert(DQ_TILE <= 32768 + TILE, "dQ staging must fit in the dS and dO buffers");
 };
 
 enum : unsigned {
   kSiteKV = 0x200, kSiteQEmpty, kSiteQFull, kSiteSFull, kSiteDpFull, kSitePFull, kSiteDsFull,
-  kSiteDqFull, kSiteDqFree, kSiteFinal, kSiteStage
+  kSiteDqFull, kSiteDqFree, kSiteFinal, kSiteStage, kSiteDoEmpty, kSiteDoFull, kSiteDsFree
 };
 
 // dQ tile layout (workspace and staging): element (row r, column d) of a 128-row tile
@@ -195,17 +203,21 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* kv_full = bars;
-  uint64_t* q_full = bars + 1;
-  uint64_t* q_empty = bars + 3;
-  uint64_t* s_full = bars + 5;
-  uint64_t* dp_full = bars + 6;
-  uint64_t* p_full = bars + 7;
-  uint64_t* ds_full = bars + 8;
-  uint64_t* dq_full = bars + 9;
-  uint64_t* dq_free = bars + 10;
-  uint64_t* dkv_final = bars + 11;
-  uint64_t* drain = bars + 12;
-  uint64_t* stage_ready = bars + 13;
+  uint64_t* q_full = bars + 1;     // [2] Q tile + LSE + Delta of a stage landed
+  uint64_t* q_empty = bars + 3;    // [2] the stage's Q buffer may be refilled
+  uint64_t* do_full = bars + 5;    // [2] dO tile landed
+  uint64_t* do_empty = bars + 7;   // [2] the stage's dO buffer may be refilled
+  uint64_t* s_full = bars + 9;
+  uint64_t* dp_full = bars + 10;
+  uint64_t* p_full = bars + 11;
+  uint64_t* ds_full = bars + 12;
+  uint64_t* dq_full = bars + 13;
+  uint64_t* dq_free = bars + 14;   // dQ columns of TMEM read out
+  uint64_t* ds_free = bars + 15;   // dS buffer (also dQ staging) may be rewritten
+  uint64_t* stage_a = bars + 16;   // dQ staging half A written (dS buffer)
+  uint64_t* stage_b = bars + 17;   // dQ staging half B written (dO buffer, D = 128)
+  uint64_t* dkv_final = bars + 18;
+  uint64_t* drain = bars + 19;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   float* lse_s = reinterpret_cast<float*>(smem + C::OFF_LSE);
@@ -217,6 +229,8 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     for (int i = 0; i < 2; ++i) {
       mbar_init(&q_full[i], 1);
       mbar_init(&q_empty[i], 1);
+      mbar_init(&do_full[i], 1);
+      mbar_init(&do_empty[i], 1);
     }
     mbar_init(s_full, 1);
     mbar_init(dp_full, 1);
@@ -224,9 +238,11 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     mbar_init(ds_full, 4);
     mbar_init(dq_full, 1);
     mbar_init(dq_free, 4);
+    mbar_init(ds_free, 1);
+    mbar_init(stage_a, 4);
+    mbar_init(stage_b, 4);
     mbar_init(dkv_final, 1);
     mbar_init(drain, 1);
-    mbar_init(stage_ready, 4);
     fence_mbar_init();
   }
   if (warp == kWarpMMA) {
@@ -245,10 +261,11 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   const uint32_t tmem = *tmem_slot;
   const WaitCtl wc{p.status, abort_flag, p.timeout_ns};
 
-  if (warp == kWarpTMA) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      int nissued = 0;
+  if (warp >= 8) {
+    reg_dealloc<kRegsControl>();
+    if (warp == kWarpTMA && lane == 0) {
+      // ---------------------------------------------------------- producer
+      int nq_issued = 0, ndo_issued = 0;
       mbar_arrive_expect_tx(kv_full, 2 * C::TILE);
       for (int hf = 0; hf < D / 64; ++hf) {
         tma_load_3d(&tm_k, kv_full, smem + C::OFF_K + hf * kSlab, hf * 64, g, start + 128 * n);
@@ -256,30 +273,34 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       }
       for (int it = 0; it < iters; ++it) {
         const int st = it & 1;
+        const uint32_t ph = ((it >> 1) & 1) ^ 1;
         const int hq = g * p.G + it / per_head;
         const int m = m0 + it % per_head;
-        if (!mbar_wait(&q_empty[st], ((it >> 1) & 1) ^ 1, wc, kSiteQEmpty)) break;
-        mbar_arrive_expect_tx(&q_full[st], 2 * C::TILE + 1024);
-        for (int hf = 0; hf < D / 64; ++hf) {
+        if (!mbar_wait(&q_empty[st], ph, wc, kSiteQEmpty)) break;
+        mbar_arrive_expect_tx(&q_full[st], C::TILE + 1024);
+        for (int hf = 0; hf < D / 64; ++hf)
           tma_load_3d(&tm_q, &q_full[st], smem + C::OFF_Q + st * C::TILE + hf * kSlab, hf * 64, hq,
                       start + 128 * m);
-          tma_load_3d(&tm_do, &q_full[st], smem + C::OFF_DO + st * C::TILE + hf * kSlab, hf * 64,
-                      hq, start + 128 * m);
-        }
         const size_t wi = (size_t(hq) * p.ntile + tile_base + m) * 128;
         bulk_load(lse_s + st * 128, p.lse2 + wi, 512, &q_full[st]);
         bulk_load(delta_s + st * 128, p.delta + wi, 512, &q_full[st]);
-        ++nissued;
+        ++nq_issued;
+        if (!mbar_wait(&do_empty[st], ph, wc, kSiteDoEmpty)) break;
+        mbar_arrive_expect_tx(&do_full[st], C::TILE);
+        for (int hf = 0; hf < D / 64; ++hf)
+          tma_load_3d(&tm_do, &do_full[st], smem + C::OFF_DO + st * C::TILE + hf * kSlab, hf * 64,
+                      hq, start + 128 * m);
+        ++ndo_issued;
       }
       mbar_drain(kv_full, 0, drain_ns(abort_flag, p.timeout_ns));
       for (int st = 0; st < 2; ++st) {
-        const int c = nissued > st ? (nissued - 1 - st) / 2 + 1 : 0;
-        if (c) mbar_drain(&q_full[st], (c - 1) & 1, drain_ns(abort_flag, p.timeout_ns));
+        const int cq = nq_issued > st ? (nq_issued - 1 - st) / 2 + 1 : 0;
+        const int cd = ndo_issued > st ? (ndo_issued - 1 - st) / 2 + 1 : 0;
+        if (cq) mbar_drain(&q_full[st], (cq - 1) & 1, drain_ns(abort_flag, p.timeout_ns));
+        if (cd) mbar_drain(&do_full[st], (cd - 1) & 1, drain_ns(abort_flag, p.timeout_ns));
       }
-    }
-  } else if (warp == kWarpMMA) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    } else if (warp == kWarpMMA && lane == 0) {
+      // ---------------------------------------------------------- MMA issuer
       constexpr uint32_t idS = idesc_bf16_f32(128, 128, 0, 0);   // S^T, dP^T
       constexpr uint32_t idKV = idesc_bf16_f32(128, D, 0, 1);    // dV, dK (A from TMEM)
       constexpr uint32_t idQ = idesc_bf16_f32(128, D, 1, 1);     // dQ (A = dS, MN-major)
@@ -302,9 +323,11 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       }
       for (int it = 0; it < iters && ok; ++it) {
         const int st = it & 1;
+        const uint32_t ph = (it >> 1) & 1;
         const uint32_t qb = smem_u32(smem + C::OFF_Q + st * C::TILE);
         const uint32_t dob = smem_u32(smem + C::OFF_DO + st * C::TILE);
         if (it > 0 && !(ok = mbar_wait(dq_free, (it - 1) & 1, wc, kSiteDqFree))) break;
+        if (!(ok = mbar_wait(&do_full[st], ph, wc, kSiteDoFull))) break;
         tc_fence_after();
         issue_T(C::COL_DP, vb, dob);  // dP^T = V dO^T
         mma_commit(dp_full);
@@ -314,6 +337,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         for (int kk = 0; kk < 8; ++kk)  // dV += P^T dO
           mma_ts(tmem + C::COL_DV, tmem + C::COL_S + kk * 8, sdesc_sw128(dob + kk * 2048, kSlab, 1024),
                  idKV, (it > 0 || kk > 0) ? 1u : 0u);
+        if (D == 64) mma_commit(&do_empty[st]);  // D = 128 stages dQ there: released by the dQ warps
         if (it + 1 < iters) {
           if (!(ok = mbar_wait(&q_full[st ^ 1], ((it + 1) >> 1) & 1, wc, kSiteQFull))) break;
           tc_fence_after();
@@ -326,17 +350,19 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         for (int kk = 0; kk < 8; ++kk)  // dK += dS^T Q
           mma_ts(tmem + C::COL_DK, tmem + C::COL_DP + kk * 8, sdesc_sw128(qb + kk * 2048, kSlab, 1024),
                  idKV, (it > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&q_empty[st]);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)  // dQ_tile = dS K
           mma_ss(tmem + C::COL_DQ, sdesc_sw128(dsb + kk * 2048, 16384, 1024),
                  sdesc_sw128(kb + kk * 2048, kSlab, 1024), idQ, kk > 0 ? 1u : 0u);
-        mma_commit(dq_full);  // the stage is released by the dQ warps after staging
+        mma_commit(dq_full);
       }
       if (ok) mma_commit(dkv_final);
       mma_commit(drain);
       mbar_drain(drain, 0, drain_ns(abort_flag, p.timeout_ns));
     }
   } else if (warp < 4) {
+    reg_alloc<kRegsCompute>();
     // ------------------------------------------------------------ P^T and dS^T
     const int qw = warp;
     const int r = qw * 32 + lane;      // key row in the tile
@@ -374,14 +400,18 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       }
       const bool diag = p.causal && m == n;
       const float4* lse4 = reinterpret_cast<const float4*>(lse_t);
+      const uint64_t cc = f2_pack(c, c);
 #pragma unroll
       for (int i4 = 0; i4 < 32; ++i4) {
         const float4 l4 = lse4[i4];
-        const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+        float x0, x1, x2, x3;
+        f2_unpack(f2_fma(f2_pack(pr[4 * i4], pr[4 * i4 + 1]), cc, f2_pack(-l4.x, -l4.y)), x0, x1);
+        f2_unpack(f2_fma(f2_pack(pr[4 * i4 + 2], pr[4 * i4 + 3]), cc, f2_pack(-l4.z, -l4.w)), x2, x3);
+        const float xv[4] = {x0, x1, x2, x3};
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           const int i = 4 * i4 + u;
-          const float e = ex2_approx(fmaf(pr[i], c, -lv[u]));
+          const float e = ex2_approx(xv[u]);
           pr[i] = (key_ok && !(diag && i < r)) ? e : 0.f;
         }
       }
@@ -398,9 +428,10 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       if (lane == 0) mbar_arrive(p_full);
 
       // dS^T = P^T * (dP^T - Delta): written in place into the dP columns (bf16) for the
-      // dK MMA and into shared memory (MN-major) for the dQ MMA.
+      // dK MMA and into shared memory (MN-major) for the dQ MMA, once the dQ warps have
+      // released that buffer (they stage the previous dQ tile in it).
       ok = __all_sync(0xffffffffu, mbar_wait(dp_full, it & 1, wc, kSiteDpFull) &&
-                                       (it == 0 || mbar_wait(dq_full, (it - 1) & 1, wc, kSiteDqFull)));
+                                       (it == 0 || mbar_wait(ds_free, (it - 1) & 1, wc, kSiteDsFree)));
       if (!ok) break;
       tc_fence_after();
 #pragma unroll
@@ -414,10 +445,15 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         for (int i4 = 0; i4 < 8; ++i4) {
           const float4 d4 = dl4[i4];
           const int c0 = ch * 32 + 4 * i4;
-          pk[2 * i4] = pack_bf16x2(pr[c0] * (__uint_as_float(u[4 * i4]) - d4.x),
-                                   pr[c0 + 1] * (__uint_as_float(u[4 * i4 + 1]) - d4.y));
-          pk[2 * i4 + 1] = pack_bf16x2(pr[c0 + 2] * (__uint_as_float(u[4 * i4 + 2]) - d4.z),
-                                       pr[c0 + 3] * (__uint_as_float(u[4 * i4 + 3]) - d4.w));
+          float a0, a1, a2, a3;
+          f2_unpack(f2_mul(f2_pack(pr[c0], pr[c0 + 1]),
+                           f2_add(f2_pack(__uint_as_float(u[4 * i4]), __uint_as_float(u[4 * i4 + 1])),
+                                  f2_pack(-d4.x, -d4.y))), a0, a1);
+          f2_unpack(f2_mul(f2_pack(pr[c0 + 2], pr[c0 + 3]),
+                           f2_add(f2_pack(__uint_as_float(u[4 * i4 + 2]), __uint_as_float(u[4 * i4 + 3])),
+                                  f2_pack(-d4.z, -d4.w))), a2, a3);
+          pk[2 * i4] = pack_bf16x2(a0, a1);
+          pk[2 * i4 + 1] = pack_bf16x2(a2, a3);
         }
         tmem_st16(tP + ch * 16, pk);
         // shared memory: query rows ch*32 .. ch*32+31 -> 64-row block ch/2, 16-byte chunks
@@ -461,14 +497,18 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       }
     }
   } else {
+    reg_alloc<kRegsCompute>();
     // ------------------------------------------------------------ dQ drain (warps 4-7)
-    // Per query tile: read dQ_tile from TMEM (thread = row), free the TMEM columns,
-    // write the rows into this stage's Q/dO buffers (the tile's MMAs are done with
-    // them) in the workspace's tile layout, then one thread issues a bulk fp32
-    // reduce-add of the whole tile into the workspace and releases the stage.
+    // Per query tile: read dQ_tile from TMEM (thread = row) and free those columns;
+    // write columns 0..63 into the dS buffer (the dQ MMA that read dS is done) and,
+    // for D = 128, columns 64..127 into this stage's dO buffer (its MMAs are done),
+    // in the workspace's tile layout; one thread bulk-reduces each half into the
+    // workspace and releases the buffers as soon as their reads complete.
     const int qw = warp & 3;
     const int r = qw * 32 + lane;      // query row of the tile (dQ) / key row (dK epilogue)
     const uint32_t tQ = tmem_addr(tmem, qw * 32, C::COL_DQ);
+    const bool leader = (qw == 0 && lane == 0);
+    constexpr int kHalfA = (C::DQ_TILE < 32768) ? C::DQ_TILE : 32768;  // bytes staged in dS buffer
     bool ok = true;
     for (int it = 0; it < iters; ++it) {
       const int st = it & 1;
@@ -489,34 +529,49 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(dq_free);
-      uint8_t* stage_q = smem + C::OFF_Q + st * C::TILE;
-      uint8_t* stage_do = smem + C::OFF_DO + st * C::TILE;
+      float* gdst = p.dq_acc + (size_t(hq) * p.ntile + tile_base + m) * 128 * D;
+      // half A: 16-byte chunks 0 .. kHalfA/2048-1 -> dS buffer
+      uint8_t* sa = smem + C::OFF_DS;
 #pragma unroll
-      for (int c4 = 0; c4 < D / 4; ++c4) {
-        uint8_t* dst = (c4 * 2048 < C::TILE) ? stage_q + c4 * 2048 : stage_do + (c4 * 2048 - C::TILE);
-        *reinterpret_cast<uint4*>(dst + r * 16) =
+      for (int c4 = 0; c4 < kHalfA / 2048; ++c4)
+        *reinterpret_cast<uint4*>(sa + c4 * 2048 + r * 16) =
             make_uint4(acc[4 * c4], acc[4 * c4 + 1], acc[4 * c4 + 2], acc[4 * c4 + 3]);
-      }
       fence_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(stage_ready);
-      if (qw == 0 && lane == 0) {
-        if (mbar_wait(stage_ready, it & 1, wc, kSiteStage)) {
-          float* dst = p.dq_acc + (size_t(hq) * p.ntile + tile_base + m) * 128 * D;
-          if (C::DQ_TILE > C::TILE) {
-            bulk_reduce_add_f32(dst, stage_q, C::TILE);
-            bulk_reduce_add_f32(dst + C::TILE / 4, stage_do, C::DQ_TILE - C::TILE);
-          } else {
-            bulk_reduce_add_f32(dst, stage_q, C::DQ_TILE);
-          }
+      if (lane == 0) mbar_arrive(stage_a);
+      if (leader) {
+        if (mbar_wait(stage_a, it & 1, wc, kSiteStage)) {
+          bulk_reduce_add_f32(gdst, sa, kHalfA);
           bulk_commit();
-          bulk_wait_read0();
-          mbar_arrive(&q_empty[st]);
         }
+      }
+      if (C::DQ_TILE > kHalfA) {
+        // half B: remaining chunks -> this stage's dO buffer
+        uint8_t* sb = smem + C::OFF_DO + st * C::TILE;
+#pragma unroll
+        for (int c4 = kHalfA / 2048; c4 < D / 4; ++c4)
+          *reinterpret_cast<uint4*>(sb + (c4 - kHalfA / 2048) * 2048 + r * 16) =
+              make_uint4(acc[4 * c4], acc[4 * c4 + 1], acc[4 * c4 + 2], acc[4 * c4 + 3]);
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(stage_b);
+        if (leader) {
+          if (mbar_wait(stage_b, it & 1, wc, kSiteStage)) {
+            bulk_reduce_add_f32(gdst + kHalfA / 4, sb, C::DQ_TILE - kHalfA);
+            bulk_commit();
+            bulk_wait_read<1>();          // half A read: the dS buffer is free
+            mbar_arrive(ds_free);
+            bulk_wait_read<0>();          // half B read: the dO buffer is free
+            mbar_arrive(&do_empty[st]);
+          }
+        }
+      } else if (leader) {
+        bulk_wait_read<0>();
+        mbar_arrive(ds_free);
       }
       __syncwarp();
     }
-    if (qw == 0 && lane == 0) bulk_wait0();
+    if (leader) bulk_wait0();
     // epilogue: dK rows (scaled)
     if (ok) {
       ok = __all_sync(0xffffffffu, mbar_wait(dkv_final, 0, wc, kSiteFinal));

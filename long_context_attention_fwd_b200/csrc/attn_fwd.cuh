@@ -12,6 +12,7 @@
 //   warp 8      TMA producer: Q tiles once, then K_j / V_j into a ring of NS stages.
 //   warp 9      MMA issuer (one thread): S_t = Q_t K_j^T (SS, fp32 in TMEM) and
 //               O_t += P_t V_j (P read from TMEM as bf16, V from shared memory).
+//   warps 10-11 idle (they complete the control warpgroup for the register split).
 //   warps 0-3   softmax for tile 0, warps 4-7 for tile 1: one thread per query row,
 //               reads S from TMEM, exp2-based online max/sum, writes P (bf16) back
 //               into the S columns, rescales O in TMEM when the running max grows by
@@ -28,9 +29,15 @@ namespace fwd {
 
 constexpr int BM = 128;                // query rows per tile
 constexpr int BN = 128;                // keys per K/V tile
-constexpr int kThreads = 320;          // 10 warps
+constexpr int kThreads = 384;          // 12 warps; warps 10-11 only complete the control warpgroup
 constexpr int kWarpTMA = 8;
 constexpr int kWarpMMA = 9;
+// Register split (setmaxnreg), as in the backward kernel: 168 at launch, 72 for the
+// control warpgroup, 216 for the two softmax warpgroups (128*72 + 256*216 = 384*168).
+constexpr int kRegsLaunch = 168;
+constexpr int kRegsControl = 72;
+constexpr int kRegsCompute = 216;
+static_assert(128 * kRegsControl + 256 * kRegsCompute <= kThreads * kRegsLaunch, "register split");
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when max grows > 2^8
 constexpr int kSlab = 128 * 128;       // one 128-row x 64-column bf16 swizzled slab (16 KB)
 
@@ -143,7 +150,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   const uint32_t tmem = *tmem_slot;
   const WaitCtl wc{p.status, abort_flag, p.timeout_ns};
 
-  if (warp == kWarpTMA) {
+  if (warp >= 8) {
+   reg_dealloc<kRegsControl>();
+   if (warp == kWarpTMA) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       int nk = 0, nv = 0;
@@ -180,7 +189,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (cv) mbar_drain(&v_full[st], (cv - 1) & 1, drain_ns(abort_flag, p.timeout_ns));
       }
     }
-  } else if (warp == kWarpMMA) {
+   } else if (warp == kWarpMMA) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16_f32(128, 128, 0, 0);
@@ -253,7 +262,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       mma_commit(drain);
       mbar_drain(drain, 0, drain_ns(abort_flag, p.timeout_ns));
     }
+   }
   } else {
+    reg_alloc<kRegsCompute>();
     // ------------------------------------------------------------ softmax + epilogue
     const int t = warp >> 2;
     const int qw = warp & 3;

@@ -103,6 +103,26 @@ attn_status device_setup(DeviceState** out, const void* ptr = nullptr) {
       e = e ? e : cudaFuncSetAttribute(selftest::umma_selftest_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, 32768 + 128 * 64 * 2 + 2048);
       e = e ? e : cudaFuncSetAttribute(selftest::umma_selftest_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, 32768 + 128 * 128 * 2 + 2048);
       if (e != cudaSuccess) return fail_cuda("cudaFuncSetAttribute", e);
+      // The kernels re-split registers between warpgroups with setmaxnreg; that is only
+      // safe when each thread starts with exactly the budget the split was sized for.
+      const void* split_kernels[4] = {
+          reinterpret_cast<const void*>(fwd::attn_fwd_kernel<64>),
+          reinterpret_cast<const void*>(fwd::attn_fwd_kernel<128>),
+          reinterpret_cast<const void*>(bwd::attn_bwd_kernel<64>),
+          reinterpret_cast<const void*>(bwd::attn_bwd_kernel<128>)};
+      const int split_regs[4] = {fwd::kRegsLaunch, fwd::kRegsLaunch, bwd::kRegsLaunch,
+                                 bwd::kRegsLaunch};
+      for (int i = 0; i < 4; ++i) {
+        cudaFuncAttributes fa;
+        if ((e = cudaFuncGetAttributes(&fa, split_kernels[i])) != cudaSuccess)
+          return fail_cuda("cudaFuncGetAttributes", e);
+        if (fa.numRegs != split_regs[i]) {
+          snprintf(g_last_error, sizeof(g_last_error),
+                   "kernel %d compiled with %d registers per thread, register split needs %d", i,
+                   fa.numRegs, split_regs[i]);
+          return ATTN_ERR_UNSUPPORTED;
+        }
+      }
     }
     d.ready = true;
   }

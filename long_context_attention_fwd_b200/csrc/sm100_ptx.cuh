@@ -142,9 +142,10 @@ __device__ __forceinline__ void bulk_reduce_add_f32(float* dst, const void* src,
 __device__ __forceinline__ void bulk_commit() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
-// Waits until the shared-memory sources of all committed bulk groups have been read.
-__device__ __forceinline__ void bulk_wait_read0() {
-  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+// Waits until at most N of the committed bulk groups still have unread shared-memory sources.
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
 }
 // Waits until all committed bulk groups have completed.
 __device__ __forceinline__ void bulk_wait0() {
@@ -286,6 +287,18 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
       "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
           smem_u32(bar))
       : "memory");
+}
+
+// ------------------------------------------------------------------ register split
+// Warpgroup-wide: every warp of a warpgroup executes the same setmaxnreg.  An
+// increase blocks until the registers are free, so the split must fit the launch.
+template <int N>
+__device__ __forceinline__ void reg_alloc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void reg_dealloc() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 // ------------------------------------------------------------------ math helpers
