@@ -200,6 +200,9 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   const int per_head = nq - m0;
   const int iters = p.G * per_head;
   const int tile_base = (start >> 7) + seq;  // workspace tile index of query tile 0
+  // Iteration order: query tiles from the last one down to m0, the group's query heads
+  // innermost.  CTAs of one wave then start on the same tile and advance in step, so
+  // the dQ tiles they reduce into (and the Q/dO tiles they read) stay in L2.
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* kv_full = bars;
@@ -274,8 +277,8 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       for (int it = 0; it < iters; ++it) {
         const int st = it & 1;
         const uint32_t ph = ((it >> 1) & 1) ^ 1;
-        const int hq = g * p.G + it / per_head;
-        const int m = m0 + it % per_head;
+        const int hq = g * p.G + it % p.G;
+        const int m = nq - 1 - it / p.G;
         if (!mbar_wait(&q_empty[st], ph, wc, kSiteQEmpty)) break;
         mbar_arrive_expect_tx(&q_full[st], C::TILE + 1024);
         for (int hf = 0; hf < D / 64; ++hf)
@@ -375,7 +378,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     bool ok = true;
     for (int it = 0; it < iters; ++it) {
       const int st = it & 1;
-      const int m = m0 + it % per_head;
+      const int m = nq - 1 - it / p.G;
       ok = __all_sync(0xffffffffu, mbar_wait(s_full, it & 1, wc, kSiteSFull) &&
                                        mbar_wait(&q_full[st], (it >> 1) & 1, wc, kSiteQFull));
       if (!ok) break;
@@ -512,8 +515,8 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     bool ok = true;
     for (int it = 0; it < iters; ++it) {
       const int st = it & 1;
-      const int hq = g * p.G + it / per_head;
-      const int m = m0 + it % per_head;
+      const int hq = g * p.G + it % p.G;
+      const int m = nq - 1 - it / p.G;
       ok = __all_sync(0xffffffffu, mbar_wait(dq_full, it & 1, wc, kSiteDqFull));
       if (!ok) break;
       tc_fence_after();

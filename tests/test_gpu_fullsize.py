@@ -4,8 +4,9 @@ sampled outputs it can compute one by one, plus properties that hold at any size
 
   * O and LSE of sampled query rows (first/last rows, tile edges, random rows);
   * dQ of sampled query rows;
-  * dK, dV of the last keys of sampled (sequence, kv head) pairs -- only the query
-    rows after them see those keys, so the oracle's cost stays small;
+  * multi-head workloads: dQ, dK, dV over two whole (sequence, head) slices;
+    grouped-query workloads: dK, dV of the last keys of sampled (sequence, kv head)
+    pairs -- only the query rows after them see those keys, so the oracle stays cheap;
   * over ALL keys of every (sequence, kv head): sum_j dV_j equals the sum of dO over
     the group's heads and rows (each probability row sums to one), and sum_j dK_j is
     zero (each row of dS sums to zero) -- both up to bf16 rounding of P and dS.
@@ -68,20 +69,34 @@ def test_full_size_sampled(idx):
     td = cu[drows[:, 0]] + drows[:, 2]
     assert rel_l2(g["dq"][td, drows[:, 1]], dq_r) <= TOL_GRAD
 
-    # ---- dK, dV of the last keys of a few (sequence, kv head) pairs
-    picks = [(len(lens) - 1, w.Hkv - 1), (0, 0)]
-    for b, gh in picks:
-        L = lens[b]
-        if L == 0:
-            continue
-        j0 = max(0, L - 160)
-        dk_r, dv_r = oracle.bwd_dkdv_range(q, k, v, do, w.causal, w.softmax_scale, b, gh, j0, L, **kw)
-        a = cu[b]
-        assert rel_l2(g["dk"][a + j0:a + L, gh], dk_r) <= TOL_GRAD
-        assert rel_l2(g["dv"][a + j0:a + L, gh], dv_r) <= TOL_GRAD
+    G = w.Hq // w.Hkv
+    if G == 1:
+        # ---- multi-head: whole (sequence, head) slices are independent problems the
+        # oracle can afford outright, so the gradient bar is checked over full slices
+        # (the stated metric is relative L2 over whole tensors; a handful of keys is a
+        # biased sample when one key dominates their norm).
+        for b, h in ((0, 0), (len(lens) - 1, w.Hq - 1)):
+            L, a = lens[b], cu[b]
+            sl = slice(a, a + L)
+            qs, ks, vs, ds = (np.ascontiguousarray(t[sl, h:h + 1]) for t in (q, k, v, do))
+            dq_r, dk_r, dv_r = oracle.bwd(qs, ks, vs, ds, w.causal, w.softmax_scale, B=1, S=L)
+            assert rel_l2(g["dq"][sl, h], dq_r[:, 0]) <= TOL_GRAD
+            assert rel_l2(g["dk"][sl, h], dk_r[:, 0]) <= TOL_GRAD
+            assert rel_l2(g["dv"][sl, h], dv_r[:, 0]) <= TOL_GRAD
+    else:
+        # ---- grouped-query: dK, dV of the last keys of a few (sequence, kv head) pairs
+        for b, gh in ((len(lens) - 1, w.Hkv - 1), (0, 0)):
+            L = lens[b]
+            if L == 0:
+                continue
+            j0 = max(0, L - 160)
+            dk_r, dv_r = oracle.bwd_dkdv_range(q, k, v, do, w.causal, w.softmax_scale, b, gh, j0, L,
+                                               **kw)
+            a = cu[b]
+            assert rel_l2(g["dk"][a + j0:a + L, gh], dk_r) <= TOL_GRAD
+            assert rel_l2(g["dv"][a + j0:a + L, gh], dv_r) <= TOL_GRAD
 
     # ---- properties over all keys
-    G = w.Hq // w.Hkv
     for b, L in enumerate(lens):
         if L == 0:
             continue
