@@ -27,7 +27,9 @@
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  All work is
  *     asynchronous on that stream; arguments are validated synchronously before
  *     anything is launched, and nothing is launched when validation fails.
- *   - The library allocates no device memory and keeps no per-call state.
+ *   - No entry point allocates device memory, and no per-call state is kept; the one
+ *     exception to "caller-owned memory" is the fixed scratch array attn_bwd_noalloc
+ *     works in, which is part of the loaded library.
  *   - A packed batch whose cu_seqlens break the rules above cannot make a kernel read
  *     or write outside the tensors (every sequence is clamped to [0, T)), but its
  *     results are undefined; attn_check_cu_seqlens validates a host copy.
@@ -81,6 +83,32 @@ attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o,
                      int Hq, int Hkv, int S, int D, int causal, float scale,
                      const int32_t* cu_seqlens, void* workspace, size_t workspace_bytes,
                      void* stream);
+
+/* Size in bytes of the scratch array attn_bwd_noalloc works in (64 MiB). */
+#define ATTN_BWD_NOALLOC_MAX_BYTES (64u << 20)
+
+/* attn_bwd for callers that cannot allocate device memory.  The pages have no
+ * counterpart: this exists for integrations that have no device allocator where they
+ * call the backward (for example a plugin interface that passes only the tensors of
+ * one operation) or whose runtime reserves all device memory up front and forbids
+ * allocating later.  Arguments are those of attn_bwd without the workspace; the
+ * caller still passes every input and output.
+ *   - The scratch is a fixed array of ATTN_BWD_NOALLOC_MAX_BYTES inside the library,
+ *     held on every GPU that loads the library until the process exits.  Problems
+ *     whose attn_bwd_workspace_size exceeds it are refused with ATTN_ERR_INVALID_ARG
+ *     (attn_last_error says why); attn_bwd with a caller workspace has no such limit.
+ *   - The first call on a device looks up the array's device address (a set-up step
+ *     done once per device, under a lock); make that first call before any stream
+ *     capture.  This function allocates nothing and frees nothing.
+ *   - All calls share the one array, and each call leaves its contents behind; the
+ *     backward rewrites everything it reads, so nothing needs clearing between calls.
+ *     Calls whose work overlaps on the GPU (different streams, or different host
+ *     threads without ordering) race on the array and corrupt each other's results:
+ *     serialise them. */
+attn_status attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                             const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                             int B, int Hq, int Hkv, int S, int D, int causal, float scale,
+                             const int32_t* cu_seqlens, void* stream);
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char* attn_strerror(attn_status status);

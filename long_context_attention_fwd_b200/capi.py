@@ -56,6 +56,8 @@ _SIGNATURES = {
     "attn_selftest_umma": (_i, [_i, _i, _vp, _vp, _fp, _vp, _fp, _vp]),
     "attn_version": (_i, []),
     "attn_last_error": (ctypes.c_char_p, []),
+    "attn_bwd_noalloc": (_i, [_vp, _vp, _vp, _vp, _fp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
+                              ctypes.c_float, _vp, _vp]),
 }
 
 
@@ -114,6 +116,12 @@ def attn_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, S, D, causal, scale,
              workspace, workspace_bytes, stream) -> int:
     return lib().attn_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, S, D, int(causal),
                           float(scale), cu_seqlens, workspace, workspace_bytes, stream)
+
+
+def attn_bwd_noalloc(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, S, D, causal, scale,
+                     cu_seqlens, stream) -> int:
+    return lib().attn_bwd_noalloc(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, S, D, int(causal),
+                                  float(scale), cu_seqlens, stream)
 
 
 def attn_device_status(stream=None):

@@ -392,3 +392,58 @@ extern "C" attn_status attn_selftest_umma(int mode, int D, const void* a, const 
         ma, mb, mode, pin, static_cast<const __nv_bfloat16*>(at), c, dev->status, to);
   return check_launch("umma_selftest_kernel launch");
 }
+
+// ------------------------------------------------------------------ backward without allocation
+// Some callers cannot hand this library a workspace: they have no device allocator at the
+// call site (a plugin interface that passes only the tensors of one operation), or their
+// runtime reserves all device memory at start-up and forbids allocation afterwards.  For
+// them attn_bwd_noalloc runs the same backward on a fixed scratch array that lives in the
+// library itself.  Every GPU that loads the library keeps this array until the process
+// exits, so its size is kept modest; problems whose workspace is larger are refused.
+static __device__ __align__(256) uint8_t g_bwd_scratch[ATTN_BWD_NOALLOC_MAX_BYTES];
+
+namespace {
+void* g_scratch_ptr[kMaxDevices] = {};  // device address of g_bwd_scratch, per device
+std::mutex g_scratch_mu;
+}  // namespace
+
+extern "C" attn_status attn_bwd_noalloc(const void* q, const void* k, const void* v,
+                                        const void* o, const float* lse, const void* dout,
+                                        void* dq, void* dk, void* dv, int B, int Hq, int Hkv,
+                                        int S, int D, int causal, float scale,
+                                        const int32_t* cu_seqlens, void* stream) {
+  const size_t need = attn_bwd_workspace_size(B, Hq, S, D, cu_seqlens);
+  if (need == 0) return ATTN_ERR_INVALID_ARG;  // the same size checks attn_bwd applies
+  if (need > size_t(ATTN_BWD_NOALLOC_MAX_BYTES)) {
+    snprintf(g_last_error, sizeof(g_last_error),
+             "attn_bwd_noalloc: workspace of %zu bytes exceeds the static scratch of %zu bytes",
+             need, size_t(ATTN_BWD_NOALLOC_MAX_BYTES));
+    return ATTN_ERR_INVALID_ARG;
+  }
+  if (!q) return ATTN_ERR_INVALID_ARG;
+  // Set-up, once per device and with that device current: the array's name is only a
+  // host-side stand-in, so its device address is looked up and cached.
+  cudaPointerAttributes attr;
+  cudaError_t e = cudaPointerGetAttributes(&attr, q);
+  if (e != cudaSuccess) return fail_cuda("cudaPointerGetAttributes", e);
+  if (attr.type != cudaMemoryTypeDevice && attr.type != cudaMemoryTypeManaged)
+    return fail_cuda("tensor pointer is not device memory", cudaErrorInvalidValue);
+  if (attr.device < 0 || attr.device >= kMaxDevices)
+    return fail_cuda("device index", cudaErrorInvalidDevice);
+  void* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (!g_scratch_ptr[attr.device]) {
+      if ((e = cudaSetDevice(attr.device)) != cudaSuccess) return fail_cuda("cudaSetDevice", e);
+      void* ptr = nullptr;
+      if ((e = cudaGetSymbolAddress(&ptr, g_bwd_scratch)) != cudaSuccess)
+        return fail_cuda("cudaGetSymbolAddress(scratch)", e);
+      g_scratch_ptr[attr.device] = ptr;
+    }
+    scratch = g_scratch_ptr[attr.device];
+  }
+  // Nothing in the scratch needs clearing: the backward's first kernel rewrites every
+  // byte the later kernels read (dQ accumulator tiles, LSE and Delta) on each call.
+  return attn_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, S, D, causal, scale, cu_seqlens,
+                  scratch, size_t(ATTN_BWD_NOALLOC_MAX_BYTES), stream);
+}
