@@ -64,6 +64,22 @@ def workload_config(w: I.Workload) -> dict:
     return cfg
 
 
+# ---------------------------------------------------------------- ranks
+def rank_workload(w: I.Workload, rank: int) -> I.Workload:
+    """The independent batch a rank processes: the same shapes, its own seed."""
+    return I.Workload(**{**w.__dict__, "seed": w.seed + 1000 * rank})
+
+
+def max_over_ranks(values, device):
+    """Element-wise max of per-rank timings (the job is as slow as its slowest rank)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x) for x in values], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
 # ---------------------------------------------------------------- clocks
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -200,7 +216,7 @@ def run_gpu(args, w: I.Workload):
     torch.cuda.set_device(dev)
 
     # Each rank owns an independent batch: seed offset by rank.
-    wr = I.Workload(**{**w.__dict__, "seed": w.seed + 1000 * rank})
+    wr = rank_workload(w, rank)
     x = I.make_inputs(wr)
     dense = wr.varlen is None
     T = wr.tokens
@@ -297,11 +313,7 @@ def run_gpu(args, w: I.Workload):
     d2h = sum(t.numel() * t.element_size() for t in (ho, hlse, hdq, hdk, hdv))
 
     # max over ranks
-    if ws > 1:
-        import torch.distributed as dist
-        tt = torch.tensor([total_ms, e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms, e2e_ms = float(tt[0]), float(tt[1])
+    total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dev)
 
     fl_f, fl_b = I.flop_fwd(wr), I.flop_bwd(wr)
     ms_step = total_ms / args.steps
