@@ -80,6 +80,32 @@ def max_over_ranks(values, device):
     return [float(x) for x in t.tolist()]
 
 
+# ---------------------------------------------------------------- ncu traffic
+KERNEL_SOURCES = ("sm100_ptx.cuh", "attn_common.cuh", "attn_fwd.cuh", "attn_bwd.cuh")
+
+
+def kernel_sources_sha1() -> str:
+    import hashlib
+    h = hashlib.sha1()
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "long_context_attention_fwd_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def measured_traffic(workload: str, kernel: str):
+    """DRAM bytes (read + write) per launch of `kernel` from the ncu capture summarised
+    in profiles/traffic.json, or None when the kernel sources changed since the capture."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        d = json.load(open(path))
+        if d.get("kernel_sources_sha1") != kernel_sources_sha1():
+            return None
+        return d["workloads"][workload][kernel]["dram_bytes_per_launch"]
+    except Exception:
+        return None
+
+
 # ---------------------------------------------------------------- clocks
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -325,13 +351,7 @@ def run_gpu(args, w: I.Workload):
     fwd_tf = fl_f / (f_ms * 1e-3) / 1e12
     bwd_tf = fl_b / (b_ms * 1e-3) / 1e12
 
-    traffic = None
-    tp = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(tp):
-        try:
-            traffic = json.load(open(tp)).get(wr.name, {}).get("attn_bwd_kernel")
-        except Exception:
-            traffic = None
+    traffic = measured_traffic(wr.name, "attn_bwd_kernel")
 
     if rank == 0:
         line = {
