@@ -19,11 +19,11 @@
 //                   Per query tile: S^T = K Q^T, dP^T = V dO^T, dV += P^T dO,
 //                   dK += dS^T Q (P^T, dS^T read from TMEM as bf16), dQ_tile = dS K
 //                   (dS staged in shared memory), and dQ_tile is reduced into the fp32
-//                   accumulator with vector atomics.  dK/dV stay deterministic.
+//                   accumulator with coalesced vector reductions.  dK/dV stay deterministic.
 //   dq_convert      dq = bf16(scale * accumulator).
 //
 // Warps: 0-3 compute P^T and dS^T (one thread per key row), 4-7 drain dQ from TMEM
-// and bulk-reduce it into the accumulator, 8 is the TMA producer, 9 issues the MMAs,
+// and reduce it into the accumulator, 8 is the TMA producer, 9 issues the MMAs,
 // 10-11 only complete the control warpgroup for the register split.
 #pragma once
 #include <cuda_bf16.h>
@@ -63,7 +63,6 @@ struct Params {
 template <int D>
 struct Cfg {
   static constexpr int TILE = 128 * D * 2;  // one 128-row bf16 tile
-  static constexpr int DQ_TILE = 128 * D * 4;  // one 128-row fp32 dQ tile
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + TILE;
   static constexpr int OFF_Q = OFF_V + TILE;        // 2 stages
@@ -73,8 +72,8 @@ struct Cfg {
   static constexpr int OFF_DELTA = OFF_LSE + 2 * 512;
   static constexpr int OFF_BAR = OFF_DELTA + 2 * 512;
   // kv_full, q_full[2], q_empty[2], do_full[2], do_empty[2], s_full, dp_full, p_full, ds_full,
-  // dq_full, dq_free, ds_free, stage_a, stage_b, dkv_final, drain
-  static constexpr int NBAR = 20;
+  // dq_full, dq_free, dkv_final, drain
+  static constexpr int NBAR = 17;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16;
   static constexpr int kMaxDyn = 232448;
@@ -83,20 +82,16 @@ struct Cfg {
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DQ = 128, COL_DV = 256, COL_DK = 256 + D;
   static_assert(SMEM_BYTES <= kMaxDyn, "shared memory budget");
-  // The fp32 dQ tile is staged in the dS buffer (32 KB) and, for D = 128, in the dO
-  // buffer of its own stage (32 KB) once the tile's MMAs are done with them.
-  static_assert(DQ_TILE <= 32768 + TILE, "dQ staging must fit in the dS and dO buffers");
 };
 
 enum : unsigned {
   kSiteKV = 0x200, kSiteQEmpty, kSiteQFull, kSiteSFull, kSiteDpFull, kSitePFull, kSiteDsFull,
-  kSiteDqFull, kSiteDqFree, kSiteFinal, kSiteStage, kSiteDoEmpty, kSiteDoFull, kSiteDsFree
+  kSiteDqFull, kSiteDqFree, kSiteFinal, kSiteDoEmpty, kSiteDoFull
 };
 
-// dQ tile layout (workspace and staging): element (row r, column d) of a 128-row tile
-// lives at float offset ((d / 4) * 128 + r) * 4 + d % 4, so the 128 threads that each
-// own one row write 16-byte chunks to consecutive addresses (no bank conflicts) and
-// the whole tile is one contiguous block for a single bulk reduction.
+// dQ tile layout (workspace): element (row r, column d) of a 128-row tile lives at float
+// offset ((d / 4) * 128 + r) * 4 + d % 4, so the 32 threads of a warp, which own 32
+// consecutive rows, reduce 16-byte chunks into 512 contiguous bytes at a time.
 __host__ __device__ constexpr size_t dq_tile_offset(int r, int d) {
   return (size_t(d >> 2) * 128 + r) * 4 + (d & 3);
 }
@@ -216,11 +211,8 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   uint64_t* ds_full = bars + 12;
   uint64_t* dq_full = bars + 13;
   uint64_t* dq_free = bars + 14;   // dQ columns of TMEM read out
-  uint64_t* ds_free = bars + 15;   // dS buffer (also dQ staging) may be rewritten
-  uint64_t* stage_a = bars + 16;   // dQ staging half A written (dS buffer)
-  uint64_t* stage_b = bars + 17;   // dQ staging half B written (dO buffer, D = 128)
-  uint64_t* dkv_final = bars + 18;
-  uint64_t* drain = bars + 19;
+  uint64_t* dkv_final = bars + 15;
+  uint64_t* drain = bars + 16;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   float* lse_s = reinterpret_cast<float*>(smem + C::OFF_LSE);
@@ -241,9 +233,6 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     mbar_init(ds_full, 4);
     mbar_init(dq_full, 1);
     mbar_init(dq_free, 4);
-    mbar_init(ds_free, 1);
-    mbar_init(stage_a, 4);
-    mbar_init(stage_b, 4);
     mbar_init(dkv_final, 1);
     mbar_init(drain, 1);
     fence_mbar_init();
@@ -340,7 +329,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         for (int kk = 0; kk < 8; ++kk)  // dV += P^T dO
           mma_ts(tmem + C::COL_DV, tmem + C::COL_S + kk * 8, sdesc_sw128(dob + kk * 2048, kSlab, 1024),
                  idKV, (it > 0 || kk > 0) ? 1u : 0u);
-        if (D == 64) mma_commit(&do_empty[st]);  // D = 128 stages dQ there: released by the dQ warps
+        mma_commit(&do_empty[st]);
         if (it + 1 < iters) {
           if (!(ok = mbar_wait(&q_full[st ^ 1], ((it + 1) >> 1) & 1, wc, kSiteQFull))) break;
           tc_fence_after();
@@ -431,10 +420,10 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       if (lane == 0) mbar_arrive(p_full);
 
       // dS^T = P^T * (dP^T - Delta): written in place into the dP columns (bf16) for the
-      // dK MMA and into shared memory (MN-major) for the dQ MMA, once the dQ warps have
-      // released that buffer (they stage the previous dQ tile in it).
+      // dK MMA and into shared memory (MN-major) for the dQ MMA, once the previous dQ MMA
+      // has finished reading that buffer.
       ok = __all_sync(0xffffffffu, mbar_wait(dp_full, it & 1, wc, kSiteDpFull) &&
-                                       (it == 0 || mbar_wait(ds_free, (it - 1) & 1, wc, kSiteDsFree)));
+                                       (it == 0 || mbar_wait(dq_full, (it - 1) & 1, wc, kSiteDqFull)));
       if (!ok) break;
       tc_fence_after();
 #pragma unroll
@@ -502,19 +491,16 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   } else {
     reg_alloc<kRegsCompute>();
     // ------------------------------------------------------------ dQ drain (warps 4-7)
-    // Per query tile: read dQ_tile from TMEM (thread = row) and free those columns;
-    // write columns 0..63 into the dS buffer (the dQ MMA that read dS is done) and,
-    // for D = 128, columns 64..127 into this stage's dO buffer (its MMAs are done),
-    // in the workspace's tile layout; one thread bulk-reduces each half into the
-    // workspace and releases the buffers as soon as their reads complete.
+    // Per query tile: read dQ_tile from TMEM (thread = row), free those columns, and
+    // add the rows into the fp32 workspace tile with vector reductions.  In the tile
+    // layout [D/4][128][4] the 32 rows of a warp are 32 consecutive 16-byte chunks, so
+    // each warp-wide reduction covers 512 contiguous bytes (four full lines), and the
+    // reductions are fire-and-forget: nothing else waits for them.
     const int qw = warp & 3;
     const int r = qw * 32 + lane;      // query row of the tile (dQ) / key row (dK epilogue)
     const uint32_t tQ = tmem_addr(tmem, qw * 32, C::COL_DQ);
-    const bool leader = (qw == 0 && lane == 0);
-    constexpr int kHalfA = (C::DQ_TILE < 32768) ? C::DQ_TILE : 32768;  // bytes staged in dS buffer
     bool ok = true;
     for (int it = 0; it < iters; ++it) {
-      const int st = it & 1;
       const int hq = g * p.G + it % p.G;
       const int m = nq - 1 - it / p.G;
       ok = __all_sync(0xffffffffu, mbar_wait(dq_full, it & 1, wc, kSiteDqFull));
@@ -532,49 +518,13 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(dq_free);
-      float* gdst = p.dq_acc + (size_t(hq) * p.ntile + tile_base + m) * 128 * D;
-      // half A: 16-byte chunks 0 .. kHalfA/2048-1 -> dS buffer
-      uint8_t* sa = smem + C::OFF_DS;
+      float4* gdst = reinterpret_cast<float4*>(p.dq_acc + (size_t(hq) * p.ntile + tile_base + m) * 128 * D);
 #pragma unroll
-      for (int c4 = 0; c4 < kHalfA / 2048; ++c4)
-        *reinterpret_cast<uint4*>(sa + c4 * 2048 + r * 16) =
-            make_uint4(acc[4 * c4], acc[4 * c4 + 1], acc[4 * c4 + 2], acc[4 * c4 + 3]);
-      fence_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(stage_a);
-      if (leader) {
-        if (mbar_wait(stage_a, it & 1, wc, kSiteStage)) {
-          bulk_reduce_add_f32(gdst, sa, kHalfA);
-          bulk_commit();
-        }
-      }
-      if (C::DQ_TILE > kHalfA) {
-        // half B: remaining chunks -> this stage's dO buffer
-        uint8_t* sb = smem + C::OFF_DO + st * C::TILE;
-#pragma unroll
-        for (int c4 = kHalfA / 2048; c4 < D / 4; ++c4)
-          *reinterpret_cast<uint4*>(sb + (c4 - kHalfA / 2048) * 2048 + r * 16) =
-              make_uint4(acc[4 * c4], acc[4 * c4 + 1], acc[4 * c4 + 2], acc[4 * c4 + 3]);
-        fence_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(stage_b);
-        if (leader) {
-          if (mbar_wait(stage_b, it & 1, wc, kSiteStage)) {
-            bulk_reduce_add_f32(gdst + kHalfA / 4, sb, C::DQ_TILE - kHalfA);
-            bulk_commit();
-            bulk_wait_read<1>();          // half A read: the dS buffer is free
-            mbar_arrive(ds_free);
-            bulk_wait_read<0>();          // half B read: the dO buffer is free
-            mbar_arrive(&do_empty[st]);
-          }
-        }
-      } else if (leader) {
-        bulk_wait_read<0>();
-        mbar_arrive(ds_free);
-      }
-      __syncwarp();
+      for (int c4 = 0; c4 < D / 4; ++c4)
+        atomicAdd(gdst + c4 * 128 + r,
+                  make_float4(__uint_as_float(acc[4 * c4]), __uint_as_float(acc[4 * c4 + 1]),
+                              __uint_as_float(acc[4 * c4 + 2]), __uint_as_float(acc[4 * c4 + 3])));
     }
-    if (leader) bulk_wait0();
     // epilogue: dK rows (scaled)
     if (ok) {
       ok = __all_sync(0xffffffffu, mbar_wait(dkv_final, 0, wc, kSiteFinal));
