@@ -44,12 +44,25 @@ def build(force: bool = False) -> str:
     return _LIB
 
 
+def use_library(path: Optional[str]) -> None:
+    """Points the bindings at another build of attn_oracle.c (the mutation tests
+    load deliberately broken copies); None restores the default library."""
+    global _lib, _LIB_OVERRIDE
+    with _lock:
+        _LIB_OVERRIDE = path
+        _lib = None
+
+
+_LIB_OVERRIDE: Optional[str] = None
+
+
 def _load():
     global _lib
     with _lock:
         if _lib is None:
-            build()
-            lib = ctypes.CDLL(_LIB)
+            if _LIB_OVERRIDE is None:
+                build()
+            lib = ctypes.CDLL(_LIB_OVERRIDE or _LIB)
             common = [ctypes.c_int] * 6 + [ctypes.c_double, _I32]
             lib.oracle_attn_fwd.argtypes = [_D, _D, _D, _D, _D] + common
             lib.oracle_attn_fwd_rows.argtypes = [_D, _D, _D] + common + [
