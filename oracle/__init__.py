@@ -11,7 +11,9 @@ function takes fp64 arrays; bf16 inputs are widened exactly with
 
 Parity status per function (pins live in tests/test_oracle_pins.py):
   fwd, fwd_rows, bwd, bwd_dq_rows, bwd_dkdv_range -- pinned by closed forms,
-  invariants, finite differences and hand-derived golden values.
+  invariants, finite differences and hand-derived golden values;
+  merge_partials -- pinned by "merging chunk partials equals attention over all keys"
+  and its special cases.
 """
 from __future__ import annotations
 
@@ -73,6 +75,9 @@ def _load():
             lib.oracle_attn_bwd_dkdv_range.argtypes = [_D] * 4 + common + [
                 ctypes.c_int] * 4 + [_D, _D]
             lib.oracle_num_threads.restype = ctypes.c_int
+            lib.oracle_merge_partials.argtypes = [ctypes.c_int, ctypes.POINTER(_D),
+                                                  ctypes.POINTER(_D), _D, _D, ctypes.c_int64,
+                                                  ctypes.c_int]
             _lib = lib
     return _lib
 
@@ -202,3 +207,23 @@ def bwd_dkdv_range(q, k, v, do, causal: bool, scale: float, b: int, g: int, j0: 
     if rc:
         raise ValueError(f"oracle_attn_bwd_dkdv_range failed ({rc})")
     return dk, dv
+
+
+def merge_partials(o_parts, lse_parts):
+    """Exact merge of partial attention results over disjoint key subsets.
+    o_parts: list of [R, D] arrays, lse_parts: list of [R] arrays -> (o [R, D], lse [R])."""
+    o_parts = [_f64(x) for x in o_parts]
+    lse_parts = [_f64(x) for x in lse_parts]
+    n = len(o_parts)
+    R, D = o_parts[0].shape
+    for a, l in zip(o_parts, lse_parts):
+        if a.shape != (R, D) or l.shape != (R,):
+            raise ValueError("partials must share shapes")
+    optrs = (_D * n)(*[_dp(a) for a in o_parts])
+    lptrs = (_D * n)(*[_dp(l) for l in lse_parts])
+    o = np.zeros((R, D), dtype=np.float64)
+    lse = np.zeros(R, dtype=np.float64)
+    rc = _load().oracle_merge_partials(n, optrs, lptrs, _dp(o), _dp(lse), R, D)
+    if rc:
+        raise ValueError(f"oracle_merge_partials failed ({rc})")
+    return o, lse

@@ -438,3 +438,39 @@ int oracle_num_threads(void) {
     return 1;
 #endif
 }
+
+/*
+ * Merge of partial attention results (page "ms-swift集成FlashAttention 2/3，长文本训练更高效", section
+ * "单靠 FlashAttention 不够？那就加上序列并行", subsection "Ring-Attention": every device
+ * accumulates partial attention over the key/value chunks that pass by).  A partial over a
+ * key subset K_p is (O_p, LSE_p) with O_p the softmax-weighted mean over K_p and LSE_p the
+ * log of its normaliser, so over the union of disjoint subsets
+ *     LSE = ln sum_p exp(LSE_p),   O = sum_p exp(LSE_p - LSE) O_p.
+ * Partials with LSE_p = -inf (no visible key) contribute nothing; if every partial is
+ * -inf the result is O = 0, LSE = -inf.
+ * o_parts: nparts arrays of [R][D]; lse_parts: nparts arrays of [R]; o: [R][D]; lse: [R].
+ */
+int oracle_merge_partials(int nparts, const double *const *o_parts, const double *const *lse_parts,
+                          double *o, double *lse, int64_t R, int D) {
+    if (nparts < 1 || R < 0 || D < 1) return 1;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < R; ++r) {
+        double m = -INFINITY;
+        for (int p = 0; p < nparts; ++p)
+            if (lse_parts[p][r] > m) m = lse_parts[p][r];
+        for (int d = 0; d < D; ++d) o[r * D + d] = 0.0;
+        if (m == -INFINITY) {
+            lse[r] = -INFINITY;
+            continue;
+        }
+        double sum = 0.0;
+        for (int p = 0; p < nparts; ++p) sum += exp(lse_parts[p][r] - m);
+        const double L = m + log(sum);
+        for (int p = 0; p < nparts; ++p) {
+            const double w = exp(lse_parts[p][r] - L);
+            for (int d = 0; d < D; ++d) o[r * D + d] += w * o_parts[p][r * D + d];
+        }
+        lse[r] = L;
+    }
+    return 0;
+}

@@ -28,6 +28,9 @@ MUTANTS = {
                         "const double ds = pij * (delta_g[(int64_t)hh * L + i] - dp);"),
     "dv_wrong_operand": ("dv_row[d] += pij * doi[d];", "dv_row[d] += pij * qi[d];"),
     "lse_without_max": ("*lse_out = m + log(sum);", "*lse_out = log(sum);"),
+    "merge_weight_unnormalised": ("const double w = exp(lse_parts[p][r] - L);",
+                                  "const double w = exp(lse_parts[p][r] - m);"),
+    "merge_lse_without_max": ("const double L = m + log(sum);", "const double L = log(sum);"),
 }
 
 
@@ -73,6 +76,22 @@ def _pin_suite() -> list:
         if abs(lse[0, 0, i] - (0.5 * float(q[i, 0] @ kk[0, 0]) + math.log(i + 1))) > 1e-12:
             failed.append("lse_closed_form")
             break
+    # merging the partials over key chunks gives the attention over all keys (partials
+    # computed here with numpy, non-causal, one chunk at a time)
+    S3, H3, D3 = 12, 2, 4
+    q, k, v = _rnd((S3, H3, D3), 11), _rnd((S3, H3, D3), 12), _rnd((S3, H3, D3), 13)
+    po, pl = [], []
+    for a, b in ((0, 5), (5, 12)):
+        s_ = 0.6 * np.einsum("ihd,jhd->hij", q, k[a:b])
+        mx = s_.max(-1, keepdims=True)
+        e = np.exp(s_ - mx)
+        po.append(np.einsum("hij,jhd->ihd", e / e.sum(-1, keepdims=True), v[a:b]).reshape(-1, D3))
+        pl.append((mx[..., 0] + np.log(e.sum(-1))).T.reshape(-1))
+    om, lm = oracle.merge_partials(po, pl)
+    of, lf = oracle.fwd(q, k, v, False, 0.6, B=1, S=S3)
+    if not (np.allclose(om.reshape(of.shape), of, atol=1e-12)
+            and np.allclose(lm.reshape(S3, H3).T, lf[0], atol=1e-12)):
+        failed.append("merge_equals_full")
     # finite differences of L = sum(dO * O)
     S2 = 5
     q, k, v, do = _rnd((S2, 2, 3), 6), _rnd((S2, 1, 3), 7), _rnd((S2, 1, 3), 8), _rnd((S2, 2, 3), 9)

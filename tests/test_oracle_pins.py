@@ -300,3 +300,50 @@ def test_rejects_bad_arguments():
         oracle.fwd(q, k, k, True, 1.0, B=1, S=4)  # Hq % Hkv != 0
     with pytest.raises(ValueError):
         oracle.fwd(np.zeros((4, 2, 2)), k, k, True, 1.0, cu_seqlens=np.array([0, 3, 2], np.int32))
+
+
+# ---------------------------------------------------------------- partial merge
+def _chunk_partials(q, k, v, bounds, scale):
+    """Non-causal attention of every query over each key chunk: the partials a ring of
+    devices holding those chunks would produce."""
+    S, H, D = q.shape
+    parts_o, parts_l = [], []
+    for a, b in bounds:
+        o = np.zeros((S, H, D))
+        lse = np.zeros((H, S))
+        for h in range(H):
+            s_ = scale * q[:, h, :] @ k[a:b, h, :].T          # [S, L]
+            m = s_.max(1, keepdims=True)
+            e = np.exp(s_ - m)
+            o[:, h, :] = (e / e.sum(1, keepdims=True)) @ v[a:b, h, :]
+            lse[h] = (m[:, 0] + np.log(e.sum(1)))
+        parts_o.append(o.reshape(S * H, D))
+        parts_l.append(lse.T.reshape(S * H))
+    return parts_o, parts_l
+
+
+def test_merge_of_key_chunks_equals_full_attention():
+    S, H, D = 40, 2, 8
+    q, k, v = rnd((S, H, D), 60), rnd((S, H, D), 61), rnd((S, H, D), 62)
+    po, pl = _chunk_partials(q, k, v, [(0, 7), (7, 25), (25, 40)], 0.4)
+    o, lse = oracle.merge_partials(po, pl)
+    of, lf = oracle.fwd(q, k, v, False, 0.4, B=1, S=S)          # oracle over all keys
+    np.testing.assert_allclose(o.reshape(S, H, D), of, atol=1e-12)
+    np.testing.assert_allclose(lse.reshape(S, H).T, lf[0], atol=1e-12)
+
+
+def test_merge_special_cases():
+    r = np.random.default_rng(3)
+    o1 = r.standard_normal((5, 4))
+    l1 = r.standard_normal(5)
+    o, l = oracle.merge_partials([o1], [l1])                   # one partial: identity
+    np.testing.assert_allclose(o, o1, atol=1e-15)
+    np.testing.assert_allclose(l, l1, atol=1e-15)
+    ninf = np.full(5, -np.inf)
+    o, l = oracle.merge_partials([o1, 7 * o1], [l1, ninf])      # -inf partial: ignored
+    np.testing.assert_allclose(o, o1, atol=1e-15)
+    o, l = oracle.merge_partials([o1, o1], [ninf, ninf])        # nothing visible
+    assert (o == 0).all() and np.isneginf(l).all()
+    o, l = oracle.merge_partials([o1, 3 * o1], [l1, l1])        # equal weights: mean
+    np.testing.assert_allclose(o, 2 * o1, atol=1e-14)
+    np.testing.assert_allclose(l, l1 + np.log(2), atol=1e-14)
