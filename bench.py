@@ -11,6 +11,10 @@ FLOP convention: forward 4*S^2*D*Hq*B, halved when causal; backward 2.5x that.
 Under torchrun (N > 1) every rank runs its own independent batch (weak scaling,
 no collective on the data path); the reported time is the max over ranks.
 
+On one GPU the line also carries "ring": the exact merge kernel of Ring attention
+(attn_merge, HBM-bound, against the measured copy bandwidth) and the forward of a
+4-rank ring run rank after rank on this GPU; both are measured after the timed steps.
+
 --impl reference times the fp64 CPU oracle (the reference arm of this build) on a
 bounded sample of the same workload: the first tokens of the causal sequence form
 an exact sub-problem, so each step runs the oracle's forward and backward on them.
@@ -228,6 +232,60 @@ def run_reference(args, w: I.Workload):
 
 
 # ---------------------------------------------------------------- GPU arm
+def ring_measurements(wr: I.Workload, q, k, v, o, lse, stream, peaks, world=4, reps=10):
+    """Measures the Ring-attention rows on one GPU, outside the timed step:
+    (1) attn_merge over `world` full-size partials (HBM-bound: bytes read + written per
+        launch / CUDA-event time, against the measured copy bandwidth);
+    (2) the forward of a `world`-rank ring run rank after rank on this GPU (chunk partials
+        from attn_fwd + attn_merge), against the single-kernel forward of the same problem.
+    Every buffer is far larger than L2, so no flush is needed between launches."""
+    import torch
+    from long_context_attention_fwd_b200 import ops, ring
+
+    o_parts = [o.clone() for _ in range(world)]
+    lse_parts = [lse + 0.25 * j for j in range(world)]
+    out, lse_out = torch.empty_like(o), torch.empty_like(lse)
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(reps)]
+        torch.cuda.synchronize()
+        for e0, e1 in evs:
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        return statistics.median(e0.elapsed_time(e1) for e0, e1 in evs)
+
+    merge_ms = timed(lambda: ops.attn_merge(o_parts, lse_parts, out=out, lse=lse_out))
+    row_bytes = o.numel() * o.element_size() + lse.numel() * lse.element_size()
+    merge_bytes = (world + 1) * row_bytes
+    hbm = float(peaks.get("hbm_gbs"))
+    gbs = merge_bytes / (merge_ms * 1e-3) / 1e9
+    ring_ms = timed(lambda: ring.ring_attn_fwd_single_device(q, k, v, world, wr.causal,
+                                                             wr.softmax_scale))
+    fwd_ms = timed(lambda: ops.attn_fwd(q, k, v, causal=wr.causal, scale=wr.softmax_scale))
+    del o_parts, lse_parts, out, lse_out
+    n_fwd = sum(len(ring.ring_schedule(r, world, wr.causal)) for r in range(world))
+    n_merge = sum(len(ring.ring_schedule(r, world, wr.causal)) > 1 for r in range(world))
+    return {
+        "merge": {"kernel": "attn_merge_kernel<%d>" % wr.D, "bound": "hbm",
+                  "workload": f"{world} partials of o {list(o.shape)} bf16 + lse {list(lse.shape)} "
+                              f"fp32 -> one (o, lse)",
+                  "ms": merge_ms, "bytes_per_launch": merge_bytes, "achieved": gbs,
+                  "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                  "peak_source": "MEASURED_PEAKS.json hbm_gbs (copy, read+write bytes)"},
+        "ring_fwd_one_gpu": {"world": world, "ms": ring_ms,
+                             "tflops": I.flop_fwd(wr) / (ring_ms * 1e-3) / 1e12,
+                             "single_kernel_fwd_ms": fwd_ms, "attn_fwd_launches": n_fwd,
+                             "attn_merge_launches": n_merge,
+                             "note": "every rank's partials and merge run one after another on "
+                                     "this GPU; the K/V transfers of a real ring are not timed"},
+    }
+
+
 def run_gpu(args, w: I.Workload):
     import torch
     from long_context_attention_fwd_b200 import ops
@@ -352,6 +410,9 @@ def run_gpu(args, w: I.Workload):
     bwd_tf = fl_b / (b_ms * 1e-3) / 1e12
 
     traffic = measured_traffic(wr.name, "attn_bwd_kernel")
+    ring_rows = None
+    if ws == 1 and dense and wr.B == 1 and wr.S % 4 == 0 and not args.no_ring:
+        ring_rows = ring_measurements(wr, q, k, v, o, lse, stream, peaks)
 
     if rank == 0:
         line = {
@@ -382,6 +443,8 @@ def run_gpu(args, w: I.Workload):
             "gpu_launches": 4 * args.steps,
             "clocks": clocks,
         }
+        if ring_rows is not None:
+            line["ring"] = ring_rows
         if ws == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(wr)
         print(json.dumps(line), flush=True)
@@ -400,6 +463,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-ring", action="store_true",
+                    help="skip the Ring-attention measurements (merge kernel, 1-GPU ring forward)")
     args = ap.parse_args()
     w = I.workload(args.workload)
     if args.impl == "reference":

@@ -110,6 +110,29 @@ attn_status attn_bwd_noalloc(const void* q, const void* k, const void* v, const 
                              int B, int Hq, int Hkv, int S, int D, int causal, float scale,
                              const int32_t* cu_seqlens, void* stream);
 
+/* Largest number of partial results one attn_merge call combines. */
+#define ATTN_MERGE_MAX_PARTS 16
+
+/* Exact merge of partial attention results for the same queries over disjoint key sets
+ * (page "ms-swift集成FlashAttention 2/3，长文本训练更高效", section "单靠 FlashAttention
+ * 不够？那就加上序列并行", subsection "Ring-Attention": K/V chunks travel around a ring of
+ * devices and each device accumulates the partial attention of its own queries; page
+ * "ms-swift支持GPU显存碎片整理提升利用率" describes the same scheme).  Each partial is the
+ * (o, lse) pair attn_fwd returns for one key chunk; per query row
+ *     lse = ln sum_p exp(lse_p),   o = sum_p exp(lse_p - lse) * o_p   (fp32, o rounded to bf16),
+ * which is the attention over the union of the chunks.  Partials with lse_p = -inf carry
+ * no weight; a row whose partials are all -inf gets o = 0, lse = -inf.
+ *   - o_parts, lse_parts: HOST arrays of nparts DEVICE pointers (1 <= nparts <=
+ *     ATTN_MERGE_MAX_PARTS); o_parts[p] is bf16 [B][S][H][D], lse_parts[p] fp32 [B][H][S]
+ *     (the dense layouts of attn_fwd; for a packed batch pass B = 1 and S = T, which is
+ *     the packed [T][H][D] / [H][T] layout).
+ *   - o, lse: outputs in the same layouts.  o may be o_parts[0] and lse may be
+ *     lse_parts[0] (in-place accumulation); any other overlap is undefined.
+ *   - D in {64, 128}; B * S * H < 2^31.  Pointers as in every entry point (o 16-byte,
+ *     lse 4-byte aligned).  The host arrays are read during the call only. */
+attn_status attn_merge(const void* const* o_parts, const float* const* lse_parts, int nparts,
+                       void* o, float* lse, int B, int H, int S, int D, void* stream);
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char* attn_strerror(attn_status status);
 

@@ -56,6 +56,7 @@ _SIGNATURES = {
     "attn_selftest_umma": (_i, [_i, _i, _vp, _vp, _fp, _vp, _fp, _vp]),
     "attn_version": (_i, []),
     "attn_last_error": (ctypes.c_char_p, []),
+    "attn_merge": (_i, [_vp, _vp, _i, _vp, _fp, _i, _i, _i, _i, _vp]),
     "attn_bwd_noalloc": (_i, [_vp, _vp, _vp, _vp, _fp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
                               ctypes.c_float, _vp, _vp]),
 }
@@ -122,6 +123,17 @@ def attn_bwd_noalloc(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, S, D, causal
                      cu_seqlens, stream) -> int:
     return lib().attn_bwd_noalloc(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, S, D, int(causal),
                                   float(scale), cu_seqlens, stream)
+
+
+def attn_merge(o_parts, lse_parts, o, lse, B, H, S, D, stream) -> int:
+    """o_parts / lse_parts: sequences of device addresses (marshalled into host arrays)."""
+    n = len(o_parts)
+    if n != len(lse_parts):
+        return ATTN_ERR_INVALID_ARG
+    oa = (ctypes.c_void_p * max(n, 1))(*o_parts)
+    la = (ctypes.c_void_p * max(n, 1))(*lse_parts)
+    return lib().attn_merge(ctypes.cast(oa, _vp), ctypes.cast(la, _vp), n, o, lse, B, H, S, D,
+                            stream)
 
 
 def attn_device_status(stream=None):

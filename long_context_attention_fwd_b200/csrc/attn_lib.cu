@@ -14,9 +14,12 @@
 #include "../../include/attn.h"
 #include "attn_bwd.cuh"
 #include "attn_fwd.cuh"
+#include "attn_merge.cuh"
 #include "umma_selftest.cuh"
 
 using namespace attn_sm100;
+
+static_assert(merge::kMaxParts == ATTN_MERGE_MAX_PARTS, "merge part limit out of sync");
 
 // Sticky device status: [0] status bits, [1] site code of the first timeout.
 static __device__ unsigned g_attn_status[2];
@@ -51,6 +54,7 @@ struct DeviceState {
   bool ready = false;
   bool sm100 = false;
   unsigned* status = nullptr;
+  unsigned merge_grid[2][merge::kVariants] = {};  // resident blocks per merge kernel (D 64/128)
 };
 std::mutex g_mu;
 DeviceState g_dev[kMaxDevices];
@@ -123,6 +127,22 @@ attn_status device_setup(DeviceState** out, const void* ptr = nullptr) {
           return ATTN_ERR_UNSUPPORTED;
         }
       }
+      // The merge kernels are grid-stride: one wave of resident blocks.
+      const void* merge_kernels[2][merge::kVariants] = {
+          {reinterpret_cast<const void*>(merge::attn_merge_kernel<64, 1, 4>),
+           reinterpret_cast<const void*>(merge::attn_merge_kernel<64, 2, 2>),
+           reinterpret_cast<const void*>(merge::attn_merge_kernel<64, 4, 1>)},
+          {reinterpret_cast<const void*>(merge::attn_merge_kernel<128, 1, 4>),
+           reinterpret_cast<const void*>(merge::attn_merge_kernel<128, 2, 2>),
+           reinterpret_cast<const void*>(merge::attn_merge_kernel<128, 4, 1>)}};
+      for (int i = 0; i < 2; ++i)
+        for (int v = 0; v < merge::kVariants; ++v) {
+          int per_sm = 0;
+          if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, merge_kernels[i][v],
+                                                                 merge::kThreads, 0)) != cudaSuccess)
+            return fail_cuda("cudaOccupancyMaxActiveBlocksPerMultiprocessor", e);
+          d.merge_grid[i][v] = unsigned(prop.multiProcessorCount) * unsigned(per_sm > 0 ? per_sm : 1);
+        }
     }
     d.ready = true;
   }
@@ -321,6 +341,55 @@ attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o,
     bwd::dq_convert_kernel<128><<<pgrid, 256, 0, s>>>(dq_acc, static_cast<__nv_bfloat16*>(dq), sv,
                                                      Hq, w.ntile, scale);
   return check_launch("dq_convert_kernel launch");
+}
+
+attn_status attn_merge(const void* const* o_parts, const float* const* lse_parts, int nparts,
+                       void* o, float* lse, int B, int H, int S, int D, void* stream) {
+  if (nparts < 1 || nparts > ATTN_MERGE_MAX_PARTS || !o_parts || !lse_parts || !o || !lse)
+    return ATTN_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || S < 1) return ATTN_ERR_INVALID_ARG;
+  const long long rows = (long long)B * S * H;
+  if (rows >= (1ll << 31)) return ATTN_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+  merge::Params p;
+  for (int j = 0; j < nparts; ++j) {
+    if (!o_parts[j] || !lse_parts[j]) return ATTN_ERR_INVALID_ARG;
+    if (!aligned(o_parts[j], 16) || !aligned(lse_parts[j], 4)) return ATTN_ERR_MISALIGNED;
+    p.o_parts[j] = static_cast<const uint4*>(o_parts[j]);
+    p.lse_parts[j] = lse_parts[j];
+  }
+  for (int j = nparts; j < merge::kMaxParts; ++j) {
+    p.o_parts[j] = nullptr;
+    p.lse_parts[j] = nullptr;
+  }
+  if (!aligned(o, 16) || !aligned(lse, 4)) return ATTN_ERR_MISALIGNED;
+  DeviceState* dev = nullptr;
+  attn_status st = device_setup(&dev, o);
+  if (st != ATTN_OK) return st;
+  p.o = static_cast<uint4*>(o);
+  p.lse = lse;
+  p.nparts = nparts;
+  p.H = unsigned(H);
+  p.S = unsigned(S);
+  p.rows = unsigned(rows);
+  const int var = merge::variant_for(nparts);
+  const unsigned rows_per_block =
+      unsigned(merge::kThreads / (D / 8)) * unsigned(merge::kVariantRows[var]);
+  const unsigned need = unsigned((rows + rows_per_block - 1) / rows_per_block);
+  const unsigned wave = dev->merge_grid[D == 64 ? 0 : 1][var];
+  const dim3 grid(need < wave ? need : wave);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const unsigned thr = merge::kThreads;
+  if (D == 64) {
+    if (var == 0) merge::attn_merge_kernel<64, 1, 4><<<grid, thr, 0, s>>>(p);
+    else if (var == 1) merge::attn_merge_kernel<64, 2, 2><<<grid, thr, 0, s>>>(p);
+    else merge::attn_merge_kernel<64, 4, 1><<<grid, thr, 0, s>>>(p);
+  } else {
+    if (var == 0) merge::attn_merge_kernel<128, 1, 4><<<grid, thr, 0, s>>>(p);
+    else if (var == 1) merge::attn_merge_kernel<128, 2, 2><<<grid, thr, 0, s>>>(p);
+    else merge::attn_merge_kernel<128, 4, 1><<<grid, thr, 0, s>>>(p);
+  }
+  return check_launch("attn_merge_kernel launch");
 }
 
 attn_status attn_device_status(void* stream, unsigned* site) {

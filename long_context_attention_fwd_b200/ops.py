@@ -4,6 +4,7 @@
     o, lse = attn_fwd(q, k, v, cu_seqlens=cu)                  # packed: q [T,Hq,D], cu int32 [n+1]
     dq, dk, dv = attn_bwd(q, k, v, o, lse, do, causal=True)
     o = attention(q, k, v, causal=True)                        # autograd-aware
+    o, lse = attn_merge([o1, o2], [lse1, lse2])                # exact merge of key-chunk partials
 
 All arithmetic runs in libattn.so; these functions only check shapes, allocate
 outputs with torch and pass raw pointers and the current CUDA stream.
@@ -11,11 +12,13 @@ outputs with torch and pass raw pointers and the current CUDA stream.
 from __future__ import annotations
 
 import math
-from typing import Optional, Tuple
+from typing import Optional, Sequence, Tuple
 
 import torch
 
 from . import capi
+
+MERGE_MAX_PARTS = 16  # ATTN_MERGE_MAX_PARTS of the C ABI
 
 
 def _stream(device) -> int:
@@ -126,3 +129,44 @@ def attention(q, k, v, causal: bool = True, scale: Optional[float] = None,
               cu_seqlens: Optional[torch.Tensor] = None) -> torch.Tensor:
     """Autograd-aware fused attention (forward and backward both in libattn.so)."""
     return _FusedAttention.apply(q, k, v, causal, scale, cu_seqlens)
+
+
+def attn_merge(o_parts: Sequence[torch.Tensor], lse_parts: Sequence[torch.Tensor],
+               out: Optional[torch.Tensor] = None,
+               lse: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Exact merge of partial attention results over disjoint key sets (Ring attention).
+
+    o_parts: bf16 [B,S,H,D] (or packed [T,H,D]); lse_parts: fp32 [B,H,S] (or [H,T]) -- the
+    outputs of attn_fwd for each key chunk.  Returns (o, lse) over the union of the chunks.
+    `out`/`lse` may be o_parts[0]/lse_parts[0] for an in-place merge.  More than
+    ATTN_MERGE_MAX_PARTS partials are merged in groups, then the groups are merged.
+    """
+    if len(o_parts) == 0 or len(o_parts) != len(lse_parts):
+        raise ValueError("need the same positive number of o and lse partials")
+    _check_inputs(*o_parts)
+    o0, l0 = o_parts[0], lse_parts[0]
+    if o0.dim() == 4:
+        B, S, H, D = o0.shape
+        lse_shape = (B, H, S)
+    elif o0.dim() == 3:
+        S, H, D = o0.shape
+        B = 1
+        lse_shape = (H, S)
+    else:
+        raise ValueError("o partials must be [B,S,H,D] or [T,H,D]")
+    for o_p, l_p in zip(o_parts, lse_parts):
+        if o_p.shape != o0.shape or o_p.device != o0.device:
+            raise ValueError("o partials differ in shape or device")
+        if tuple(l_p.shape) != lse_shape or l_p.dtype != torch.float32 or not l_p.is_contiguous() \
+                or l_p.device != o0.device:
+            raise ValueError(f"lse partials must be contiguous fp32 {lse_shape} on {o0.device}")
+    if len(o_parts) > MERGE_MAX_PARTS:
+        groups = [attn_merge(o_parts[i:i + MERGE_MAX_PARTS], lse_parts[i:i + MERGE_MAX_PARTS])
+                  for i in range(0, len(o_parts), MERGE_MAX_PARTS)]
+        return attn_merge([g[0] for g in groups], [g[1] for g in groups], out, lse)
+    out = torch.empty_like(o0) if out is None else out
+    lse = torch.empty_like(l0) if lse is None else lse
+    st = capi.attn_merge([t.data_ptr() for t in o_parts], [t.data_ptr() for t in lse_parts],
+                         out.data_ptr(), lse.data_ptr(), B, H, S, D, _stream(o0.device))
+    capi.check(st, "attn_merge")
+    return out, lse

@@ -80,3 +80,18 @@ def test_ops_refuses_cpu_tensors():
     q = torch.zeros(1, 128, 2, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         ops.attn_fwd(q, q, q)
+
+
+def test_merge_validation():
+    m = capi.attn_merge
+    assert m([], [], A, A, 1, 2, 8, 64, None) == capi.ATTN_ERR_INVALID_ARG          # no partials
+    assert m([A] * 17, [A] * 17, A, A, 1, 2, 8, 64, None) == capi.ATTN_ERR_INVALID_ARG
+    assert m([A, A], [A], A, A, 1, 2, 8, 64, None) == capi.ATTN_ERR_INVALID_ARG     # counts differ
+    assert m([A, None], [A, A], A, A, 1, 2, 8, 64, None) == capi.ATTN_ERR_INVALID_ARG
+    assert m([A, A], [A, A], None, A, 1, 2, 8, 64, None) == capi.ATTN_ERR_INVALID_ARG
+    assert m([A, A], [A, A], A, A, 0, 2, 8, 64, None) == capi.ATTN_ERR_INVALID_ARG  # B = 0
+    assert m([A, A], [A, A], A, A, 1, 2, 8, 96, None) == capi.ATTN_ERR_UNSUPPORTED  # D
+    assert m([A, A], [A, A], A, A, 1 << 16, 1 << 8, 1 << 8, 64, None) == capi.ATTN_ERR_INVALID_ARG
+    assert m([A, A + 8], [A, A], A, A, 1, 2, 8, 64, None) == capi.ATTN_ERR_MISALIGNED
+    assert m([A, A], [A, A + 2], A, A, 1, 2, 8, 64, None) == capi.ATTN_ERR_MISALIGNED
+    assert m([A, A], [A, A], A + 8, A, 1, 2, 8, 64, None) == capi.ATTN_ERR_MISALIGNED
