@@ -85,7 +85,7 @@ def max_over_ranks(values, device):
 
 
 # ---------------------------------------------------------------- ncu traffic
-KERNEL_SOURCES = ("sm100_ptx.cuh", "attn_common.cuh", "attn_fwd.cuh", "attn_bwd.cuh")
+KERNEL_SOURCES = ("sm100_ptx.cuh", "attn_common.cuh", "attn_fwd.cuh", "attn_bwd.cuh", "attn_merge.cuh")
 
 
 def kernel_sources_sha1() -> str:
@@ -271,11 +271,13 @@ def ring_measurements(wr: I.Workload, q, k, v, o, lse, stream, peaks, world=4, r
     n_fwd = sum(len(ring.ring_schedule(r, world, wr.causal)) for r in range(world))
     n_merge = sum(len(ring.ring_schedule(r, world, wr.causal)) > 1 for r in range(world))
     return {
-        "merge": {"kernel": "attn_merge_kernel<%d>" % wr.D, "bound": "hbm",
+        "merge": {"kernel": "attn_merge_kernel<%d,4,1>" % wr.D, "bound": "hbm",
                   "workload": f"{world} partials of o {list(o.shape)} bf16 + lse {list(lse.shape)} "
                               f"fp32 -> one (o, lse)",
                   "ms": merge_ms, "bytes_per_launch": merge_bytes, "achieved": gbs,
                   "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                  "traffic": (measured_traffic(wr.name, "attn_merge_kernel_4parts")
+                              if world == 4 else None),
                   "peak_source": "MEASURED_PEAKS.json hbm_gbs (copy, read+write bytes)"},
         "ring_fwd_one_gpu": {"world": world, "ms": ring_ms,
                              "tflops": I.flop_fwd(wr) / (ring_ms * 1e-3) / 1e12,
