@@ -13,7 +13,9 @@ no collective on the data path); the reported time is the max over ranks.
 
 On one GPU the line also carries "ring": the exact merge kernel of Ring attention
 (attn_merge, HBM-bound, against the measured copy bandwidth) and the forward of a
-4-rank ring run rank after rank on this GPU; both are measured after the timed steps.
+4-rank ring run rank after rank on this GPU; and "ulysses": the relayout kernel around
+the Ulysses all-to-alls (HBM-bound) and forward + backward of a 4-rank Ulysses group run
+rank after rank on this GPU.  All are measured after the timed steps.
 
 --impl reference times the fp64 CPU oracle (the reference arm of this build) on a
 bounded sample of the same workload: the first tokens of the causal sequence form
@@ -85,7 +87,8 @@ def max_over_ranks(values, device):
 
 
 # ---------------------------------------------------------------- ncu traffic
-KERNEL_SOURCES = ("sm100_ptx.cuh", "attn_common.cuh", "attn_fwd.cuh", "attn_bwd.cuh", "attn_merge.cuh")
+KERNEL_SOURCES = ("sm100_ptx.cuh", "attn_common.cuh", "attn_fwd.cuh", "attn_bwd.cuh",
+                  "attn_merge.cuh")
 
 
 def kernel_sources_sha1() -> str:
@@ -288,6 +291,61 @@ def ring_measurements(wr: I.Workload, q, k, v, o, lse, stream, peaks, world=4, r
     }
 
 
+def ulysses_measurements(wr: I.Workload, q, k, v, do, stream, peaks, world=4, reps=10):
+    """Measures the Ulysses rows on one GPU, outside the timed step:
+    (1) the relayout kernel (attn_transpose_blocks) on q as one rank's send buffer for a
+        `world`-rank group (HBM-bound: bytes read + written / CUDA-event time);
+    (2) forward + backward of every rank of a `world`-rank group run one after another on
+        this GPU (relayouts around emulated all-to-alls, attention per head group), beside
+        the unsplit forward + backward."""
+    import torch
+    from long_context_attention_fwd_b200 import ops
+    from long_context_attention_fwd_b200 import ulysses as U
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(reps)]
+        torch.cuda.synchronize()
+        for e0, e1 in evs:
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        return statistics.median(e0.elapsed_time(e1) for e0, e1 in evs)
+
+    B, S, Hq, D = q.shape
+    out = torch.empty_like(q)
+    tr_ms = timed(lambda: ops.transpose_blocks(q, B * S, world, out=out))
+    tr_bytes = 2 * q.numel() * q.element_size()
+    hbm = float(peaks.get("hbm_gbs"))
+    gbs = tr_bytes / (tr_ms * 1e-3) / 1e9
+    del out
+    uly_ms = timed(lambda: U.ulysses_attention_single_device(q, k, v, world, wr.causal,
+                                                             wr.softmax_scale, do=do))
+
+    def plain():
+        o, lse = ops.attn_fwd(q, k, v, causal=wr.causal, scale=wr.softmax_scale)
+        ops.attn_bwd(q, k, v, o, lse, do, causal=wr.causal, scale=wr.softmax_scale)
+
+    plain_ms = timed(plain)
+    return {
+        "relayout": {"kernel": "transpose_blocks_kernel", "bound": "hbm",
+                     "workload": f"q {list(q.shape)} bf16 -> send buffer of {world} head "
+                                 f"groups [{world}, {B * S}, {Hq // world}, {D}]",
+                     "ms": tr_ms, "bytes_per_launch": tr_bytes, "achieved": gbs, "peak": hbm,
+                     "unit": "GB/s", "frac": gbs / hbm,
+                     "peak_source": "MEASURED_PEAKS.json hbm_gbs (copy, read+write bytes)"},
+        "ulysses_fwd_bwd_one_gpu": {
+            "world": world, "ms": uly_ms,
+            "tflops": (I.flop_fwd(wr) + I.flop_bwd(wr)) / (uly_ms * 1e-3) / 1e12,
+            "unsplit_fwd_bwd_ms": plain_ms,
+            "note": "every rank's relayouts and head-group attention run one after another on "
+                    "this GPU; the all-to-alls are plain copies here, NCCL in a real group"},
+    }
+
+
 def run_gpu(args, w: I.Workload):
     import torch
     from long_context_attention_fwd_b200 import ops
@@ -412,9 +470,12 @@ def run_gpu(args, w: I.Workload):
     bwd_tf = fl_b / (b_ms * 1e-3) / 1e12
 
     traffic = measured_traffic(wr.name, "attn_bwd_kernel")
-    ring_rows = None
+    ring_rows = uly_rows = None
     if ws == 1 and dense and wr.B == 1 and wr.S % 4 == 0 and not args.no_ring:
         ring_rows = ring_measurements(wr, q, k, v, o, lse, stream, peaks)
+    if (ws == 1 and dense and wr.S % 4 == 0 and wr.Hq % 4 == 0 and wr.Hkv % 4 == 0
+            and not args.no_ulysses):
+        uly_rows = ulysses_measurements(wr, q, k, v, do, stream, peaks)
 
     if rank == 0:
         line = {
@@ -447,6 +508,8 @@ def run_gpu(args, w: I.Workload):
         }
         if ring_rows is not None:
             line["ring"] = ring_rows
+        if uly_rows is not None:
+            line["ulysses"] = uly_rows
         if ws == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(wr)
         print(json.dumps(line), flush=True)
@@ -465,6 +528,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-ulysses", action="store_true",
+                    help="skip the Ulysses measurements (relayout kernel, 1-GPU Ulysses step)")
     ap.add_argument("--no-ring", action="store_true",
                     help="skip the Ring-attention measurements (merge kernel, 1-GPU ring forward)")
     args = ap.parse_args()

@@ -133,6 +133,24 @@ attn_status attn_bwd_noalloc(const void* q, const void* k, const void* v, const 
 attn_status attn_merge(const void* const* o_parts, const float* const* lse_parts, int nparts,
                        void* o, float* lse, int B, int H, int S, int D, void* stream);
 
+/* Block transpose for the layout changes around the all-to-alls of Ulysses sequence
+ * parallelism (page "ms-swift集成FlashAttention 2/3，长文本训练更高效", section "单靠
+ * FlashAttention 不够？那就加上序列并行", Ulysses subsection: split the sequence across
+ * devices, all-to-all, attention on every device, all-to-all back to restore the order;
+ * also page "ms-swift长文本训练秘诀：Ulysses并行技术解析", section 1).  An all-to-all sends
+ * contiguous chunk p to rank p, so data bound for one rank is gathered into one chunk
+ * before the exchange and interleaved back after it:
+ *     `in` is a grid [n_outer][n_inner] of blocks of block_bytes bytes,
+ *     `out` is the grid [n_inner][n_outer]:  out[j][i] = in[i][j].
+ * Example: q of one rank, [B*C][Hq][D] bf16, seen as [B*C][N][Hq/N * D * 2 bytes] becomes
+ * the send buffer [N][B*C][Hq/N][D] (chunk p = the heads of rank p).
+ *   - in, out: DEVICE pointers, 16-byte aligned, not overlapping (INVALID_ARG if they do);
+ *     block_bytes a multiple of 16 (MISALIGNED otherwise) and >= 16;
+ *     n_outer * n_inner * block_bytes / 16 < 2^31.
+ *   - A pure copy: bit-exact, no arithmetic. */
+attn_status attn_transpose_blocks(const void* in, void* out, long long n_outer, long long n_inner,
+                                  long long block_bytes, void* stream);
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char* attn_strerror(attn_status status);
 

@@ -56,6 +56,8 @@ _SIGNATURES = {
     "attn_selftest_umma": (_i, [_i, _i, _vp, _vp, _fp, _vp, _fp, _vp]),
     "attn_version": (_i, []),
     "attn_last_error": (ctypes.c_char_p, []),
+    "attn_transpose_blocks": (_i, [_vp, _vp, ctypes.c_longlong, ctypes.c_longlong,
+                                   ctypes.c_longlong, _vp]),
     "attn_merge": (_i, [_vp, _vp, _i, _vp, _fp, _i, _i, _i, _i, _vp]),
     "attn_bwd_noalloc": (_i, [_vp, _vp, _vp, _vp, _fp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
                               ctypes.c_float, _vp, _vp]),
@@ -134,6 +136,11 @@ def attn_merge(o_parts, lse_parts, o, lse, B, H, S, D, stream) -> int:
     la = (ctypes.c_void_p * max(n, 1))(*lse_parts)
     return lib().attn_merge(ctypes.cast(oa, _vp), ctypes.cast(la, _vp), n, o, lse, B, H, S, D,
                             stream)
+
+
+def attn_transpose_blocks(inp, out, n_outer, n_inner, block_bytes, stream) -> int:
+    return lib().attn_transpose_blocks(inp, out, int(n_outer), int(n_inner), int(block_bytes),
+                                       stream)
 
 
 def attn_device_status(stream=None):

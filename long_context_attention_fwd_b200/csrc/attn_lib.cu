@@ -15,6 +15,7 @@
 #include "attn_bwd.cuh"
 #include "attn_fwd.cuh"
 #include "attn_merge.cuh"
+#include "attn_relayout.cuh"
 #include "umma_selftest.cuh"
 
 using namespace attn_sm100;
@@ -55,6 +56,7 @@ struct DeviceState {
   bool sm100 = false;
   unsigned* status = nullptr;
   unsigned merge_grid[2][merge::kVariants] = {};  // resident blocks per merge kernel (D 64/128)
+  unsigned relayout_grid = 0;                     // resident blocks of transpose_blocks_kernel
 };
 std::mutex g_mu;
 DeviceState g_dev[kMaxDevices];
@@ -143,6 +145,13 @@ attn_status device_setup(DeviceState** out, const void* ptr = nullptr) {
             return fail_cuda("cudaOccupancyMaxActiveBlocksPerMultiprocessor", e);
           d.merge_grid[i][v] = unsigned(prop.multiProcessorCount) * unsigned(per_sm > 0 ? per_sm : 1);
         }
+      {
+        int per_sm = 0;
+        if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+                 &per_sm, relayout::transpose_blocks_kernel, relayout::kThreads, 0)) != cudaSuccess)
+          return fail_cuda("cudaOccupancyMaxActiveBlocksPerMultiprocessor", e);
+        d.relayout_grid = unsigned(prop.multiProcessorCount) * unsigned(per_sm > 0 ? per_sm : 1);
+      }
     }
     d.ready = true;
   }
@@ -390,6 +399,36 @@ attn_status attn_merge(const void* const* o_parts, const float* const* lse_parts
     else merge::attn_merge_kernel<128, 4, 1><<<grid, thr, 0, s>>>(p);
   }
   return check_launch("attn_merge_kernel launch");
+}
+
+attn_status attn_transpose_blocks(const void* in, void* out, long long n_outer, long long n_inner,
+                                  long long block_bytes, void* stream) {
+  if (!in || !out || n_outer < 1 || n_inner < 1 || block_bytes < 16) return ATTN_ERR_INVALID_ARG;
+  if (block_bytes % 16) return ATTN_ERR_MISALIGNED;
+  if (!aligned(in, 16) || !aligned(out, 16)) return ATTN_ERR_MISALIGNED;
+  const long long vec = block_bytes / 16;
+  if (n_outer >= (1ll << 31) || n_inner >= (1ll << 31) || vec >= (1ll << 31) ||
+      (double)n_outer * (double)n_inner * (double)vec >= 2147483648.0)
+    return ATTN_ERR_INVALID_ARG;
+  const long long total = n_outer * n_inner * vec;
+  const uintptr_t a = reinterpret_cast<uintptr_t>(in), b = reinterpret_cast<uintptr_t>(out);
+  const uintptr_t span = uintptr_t(total) * 16;
+  if (a < b + span && b < a + span) return ATTN_ERR_INVALID_ARG;  // in and out overlap
+  DeviceState* dev = nullptr;
+  attn_status st = device_setup(&dev, in);
+  if (st != ATTN_OK) return st;
+  relayout::Params p;
+  p.in = static_cast<const uint4*>(in);
+  p.out = static_cast<uint4*>(out);
+  p.n_outer = unsigned(n_outer);
+  p.n_inner = unsigned(n_inner);
+  p.vec = unsigned(vec);
+  p.total = unsigned(total);
+  const long long per_pass = (long long)relayout::kThreads * relayout::kUnroll;
+  const unsigned need = unsigned((total + per_pass - 1) / per_pass);
+  const dim3 grid(need < dev->relayout_grid ? need : dev->relayout_grid);
+  relayout::transpose_blocks_kernel<<<grid, relayout::kThreads, 0, static_cast<cudaStream_t>(stream)>>>(p);
+  return check_launch("transpose_blocks_kernel launch");
 }
 
 attn_status attn_device_status(void* stream, unsigned* site) {

@@ -170,3 +170,24 @@ def attn_merge(o_parts: Sequence[torch.Tensor], lse_parts: Sequence[torch.Tensor
                          out.data_ptr(), lse.data_ptr(), B, H, S, D, _stream(o0.device))
     capi.check(st, "attn_merge")
     return out, lse
+
+
+def transpose_blocks(x: torch.Tensor, n_outer: int, n_inner: int,
+                     out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """x seen as [n_outer][n_inner][block] -> [n_inner][n_outer][block] (a copy in
+    libattn.so; the block is x.numel() / (n_outer * n_inner) elements).  Returns a tensor
+    of x's dtype and shape [n_inner, n_outer, block] unless `out` is given."""
+    if not x.is_cuda or not x.is_contiguous():
+        raise ValueError("transpose_blocks needs a contiguous CUDA tensor (there is no CPU path)")
+    n = x.numel()
+    if n_outer < 1 or n_inner < 1 or n % (n_outer * n_inner):
+        raise ValueError("x does not split into n_outer * n_inner equal blocks")
+    blk = n // (n_outer * n_inner)
+    if out is None:
+        out = torch.empty((n_inner, n_outer, blk), dtype=x.dtype, device=x.device)
+    elif out.numel() != n or not out.is_contiguous() or out.dtype != x.dtype:
+        raise ValueError("out must be contiguous, of x's dtype and size")
+    st = capi.attn_transpose_blocks(x.data_ptr(), out.data_ptr(), n_outer, n_inner,
+                                    blk * x.element_size(), _stream(x.device))
+    capi.check(st, "attn_transpose_blocks")
+    return out

@@ -95,3 +95,14 @@ def test_merge_validation():
     assert m([A, A + 8], [A, A], A, A, 1, 2, 8, 64, None) == capi.ATTN_ERR_MISALIGNED
     assert m([A, A], [A, A + 2], A, A, 1, 2, 8, 64, None) == capi.ATTN_ERR_MISALIGNED
     assert m([A, A], [A, A], A + 8, A, 1, 2, 8, 64, None) == capi.ATTN_ERR_MISALIGNED
+
+
+def test_transpose_blocks_validation():
+    t = capi.attn_transpose_blocks
+    assert t(None, A, 2, 2, 16, None) == capi.ATTN_ERR_INVALID_ARG
+    assert t(A, A + (1 << 20), 0, 2, 16, None) == capi.ATTN_ERR_INVALID_ARG      # n_outer = 0
+    assert t(A, A + (1 << 20), 2, 2, 8, None) == capi.ATTN_ERR_INVALID_ARG       # < 16 bytes
+    assert t(A, A + (1 << 20), 2, 2, 24, None) == capi.ATTN_ERR_MISALIGNED       # not 16k bytes
+    assert t(A + 8, A + (1 << 20), 2, 2, 16, None) == capi.ATTN_ERR_MISALIGNED
+    assert t(A, A + 32, 2, 2, 16, None) == capi.ATTN_ERR_INVALID_ARG             # overlap
+    assert t(A, A + (1 << 40), 1 << 20, 1 << 8, 1 << 10, None) == capi.ATTN_ERR_INVALID_ARG
