@@ -13,7 +13,9 @@ Parity status per function (pins live in tests/test_oracle_pins.py):
   fwd, fwd_rows, bwd, bwd_dq_rows, bwd_dkdv_range -- pinned by closed forms,
   invariants, finite differences and hand-derived golden values;
   merge_partials -- pinned by "merging chunk partials equals attention over all keys"
-  and its special cases.
+  and its special cases;
+  decode -- pinned by PyTorch's fp64 attention routine, closed forms (V = ones, identical
+  keys, one cached key, an empty cache) and grouped-query = repeated multi-head.
 """
 from __future__ import annotations
 
@@ -75,6 +77,9 @@ def _load():
             lib.oracle_attn_bwd_dkdv_range.argtypes = [_D] * 4 + common + [
                 ctypes.c_int] * 4 + [_D, _D]
             lib.oracle_num_threads.restype = ctypes.c_int
+            lib.oracle_attn_decode.argtypes = [_D, _D, _D, _I32, _D, _D, ctypes.c_int,
+                                               ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                               ctypes.c_int, ctypes.c_double]
             lib.oracle_merge_partials.argtypes = [ctypes.c_int, ctypes.POINTER(_D),
                                                   ctypes.POINTER(_D), _D, _D, ctypes.c_int64,
                                                   ctypes.c_int]
@@ -226,4 +231,24 @@ def merge_partials(o_parts, lse_parts):
     rc = _load().oracle_merge_partials(n, optrs, lptrs, _dp(o), _dp(lse), R, D)
     if rc:
         raise ValueError(f"oracle_merge_partials failed ({rc})")
+    return o, lse
+
+
+def decode(q, k_cache, v_cache, cache_len, scale: float):
+    """Decode attention: q [B,Hq,D], k/v cache [B,Lmax,Hkv,D], cache_len [B] ->
+    (o [B,Hq,D], lse [B,Hq])."""
+    q, k_cache, v_cache = _f64(q), _f64(k_cache), _f64(v_cache)
+    B, Hq, D = q.shape
+    _, Lmax, Hkv, _ = k_cache.shape
+    if k_cache.shape != (B, Lmax, Hkv, D) or v_cache.shape != k_cache.shape:
+        raise ValueError("cache shapes must be [B, Lmax, Hkv, D]")
+    cl = np.ascontiguousarray(cache_len, dtype=np.int32)
+    if cl.shape != (B,):
+        raise ValueError("cache_len must have B entries")
+    o = np.zeros((B, Hq, D), dtype=np.float64)
+    lse = np.zeros((B, Hq), dtype=np.float64)
+    rc = _load().oracle_attn_decode(_dp(q), _dp(k_cache), _dp(v_cache), _ip(cl), _dp(o), _dp(lse),
+                                    B, Hq, Hkv, Lmax, D, float(scale))
+    if rc:
+        raise ValueError(f"oracle_attn_decode failed ({rc})")
     return o, lse

@@ -474,3 +474,67 @@ int oracle_merge_partials(int nparts, const double *const *o_parts, const double
     }
     return 0;
 }
+
+/*
+ * Decode attention over a key/value cache (page "ms-swift长文本训练秘诀：Ulysses并行技术解析",
+ * section 5 on deploying the fine-tuned model for 32K-context inference; the computation is
+ * the standard attention of page "ms-swift集成FlashAttention 2/3，长文本训练更高效", section
+ * "为什么传统注意力这么'吃'显存", for one new query token).  Sequence b has one query token
+ * q[b] (all Hq heads) and cache_len[b] cached keys/values; the new token attends to every
+ * cached key (it is the last position, so the causal mask hides nothing):
+ *     s_j = scale * q_bh . k_bjg,  P = softmax_j(s),  o_bh = sum_j P_j v_bjg,
+ *     lse_bh = ln sum_j exp(s_j),  g = h / (Hq/Hkv).
+ * cache_len[b] = 0 gives o = 0 and lse = -inf (nothing to attend to).
+ * Layouts: q, o [B][Hq][D]; k_cache, v_cache [B][Lmax][Hkv][D]; lse [B][Hq].
+ */
+int oracle_attn_decode(const double *q, const double *k_cache, const double *v_cache,
+                       const int32_t *cache_len, double *o, double *lse, int B, int Hq, int Hkv,
+                       int Lmax, int D, double scale) {
+    if (B < 1 || Hq < 1 || Hkv < 1 || Lmax < 0 || D < 1 || Hq % Hkv) return 1;
+    for (int b = 0; b < B; ++b)
+        if (cache_len[b] < 0 || cache_len[b] > Lmax) return 1;
+    const int G = Hq / Hkv;
+    int err = 0;
+#pragma omp parallel
+    {
+        double *s = (double *)malloc(sizeof(double) * (Lmax > 0 ? Lmax : 1));
+        if (!s) {
+#pragma omp atomic write
+            err = 2;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t r = 0; r < (int64_t)B * Hq; ++r) {
+            if (!s) continue;
+            const int b = (int)(r / Hq), h = (int)(r % Hq), g = h / G;
+            const int L = cache_len[b];
+            const double *qi = q + r * D;
+            double *orow = o + r * D;
+            for (int d = 0; d < D; ++d) orow[d] = 0.0;
+            if (L == 0) {
+                lse[r] = -INFINITY;
+                continue;
+            }
+            double m = -INFINITY;
+            for (int j = 0; j < L; ++j) {
+                const double *kj = k_cache + (((int64_t)b * Lmax + j) * Hkv + g) * D;
+                double acc = 0.0;
+                for (int d = 0; d < D; ++d) acc += qi[d] * kj[d];
+                s[j] = scale * acc;
+                if (s[j] > m) m = s[j];
+            }
+            double sum = 0.0;
+            for (int j = 0; j < L; ++j) {
+                s[j] = exp(s[j] - m);
+                sum += s[j];
+            }
+            for (int j = 0; j < L; ++j) {
+                const double pj = s[j] / sum;
+                const double *vj = v_cache + (((int64_t)b * Lmax + j) * Hkv + g) * D;
+                for (int d = 0; d < D; ++d) orow[d] += pj * vj[d];
+            }
+            lse[r] = m + log(sum);
+        }
+        free(s);
+    }
+    return err;
+}

@@ -31,6 +31,9 @@ MUTANTS = {
     "merge_weight_unnormalised": ("const double w = exp(lse_parts[p][r] - L);",
                                   "const double w = exp(lse_parts[p][r] - m);"),
     "merge_lse_without_max": ("const double L = m + log(sum);", "const double L = log(sum);"),
+    "decode_drops_last_key": ("const int L = cache_len[b];", "const int L = cache_len[b] > 1 ? cache_len[b] - 1 : cache_len[b];"),
+    "decode_gqa_map_modulo": ("const int b = (int)(r / Hq), h = (int)(r % Hq), g = h / G;",
+                              "const int b = (int)(r / Hq), h = (int)(r % Hq), g = h % Hkv;"),
 }
 
 
@@ -92,6 +95,20 @@ def _pin_suite() -> list:
     if not (np.allclose(om.reshape(of.shape), of, atol=1e-12)
             and np.allclose(lm.reshape(S3, H3).T, lf[0], atol=1e-12)):
         failed.append("merge_equals_full")
+    # decode: one query over a cache equals the oracle's causal attention for the last
+    # row of a sequence whose last query is that token (computed here directly in numpy)
+    Lc, Hq4, Hkv4, D4 = 9, 4, 2, 4
+    qd, kc, vc = _rnd((1, Hq4, D4), 21), _rnd((1, Lc, Hkv4, D4), 22), _rnd((1, Lc, Hkv4, D4), 23)
+    od, ld = oracle.decode(qd, kc, vc, np.array([Lc], dtype=np.int32), 0.8)
+    ok = True
+    for h in range(Hq4):
+        g = h // (Hq4 // Hkv4)
+        s_ = 0.8 * kc[0, :, g] @ qd[0, h]
+        e = np.exp(s_ - s_.max())
+        ok &= np.allclose(od[0, h], (e / e.sum()) @ vc[0, :, g], atol=1e-12)
+        ok &= abs(ld[0, h] - (s_.max() + np.log(e.sum()))) < 1e-12
+    if not ok:
+        failed.append("decode_direct")
     # finite differences of L = sum(dO * O)
     S2 = 5
     q, k, v, do = _rnd((S2, 2, 3), 6), _rnd((S2, 1, 3), 7), _rnd((S2, 1, 3), 8), _rnd((S2, 2, 3), 9)

@@ -347,3 +347,66 @@ def test_merge_special_cases():
     o, l = oracle.merge_partials([o1, 3 * o1], [l1, l1])        # equal weights: mean
     np.testing.assert_allclose(o, 2 * o1, atol=1e-14)
     np.testing.assert_allclose(l, l1 + np.log(2), atol=1e-14)
+
+
+# ---------------------------------------------------------------- decode over a cache
+def _decode_problem(B, Hq, Hkv, Lmax, D, seed):
+    q = rnd((B, Hq, D), seed)
+    k = rnd((B, Lmax, Hkv, D), seed + 1)
+    v = rnd((B, Lmax, Hkv, D), seed + 2)
+    return q, k, v
+
+
+def test_decode_matches_torch_sdpa():
+    torch = pytest.importorskip("torch")
+    B, Hq, Hkv, Lmax, D = 3, 6, 2, 23, 8
+    q, k, v = _decode_problem(B, Hq, Hkv, Lmax, D, 70)
+    lens = np.array([23, 1, 9], dtype=np.int32)
+    o, lse = oracle.decode(q, k, v, lens, 0.45)
+    G = Hq // Hkv
+    for b in range(B):
+        L = lens[b]
+        for h in range(Hq):
+            qt = torch.from_numpy(q[b, h]).view(1, 1, 1, D)
+            kt = torch.from_numpy(k[b, :L, h // G]).view(1, 1, L, D)
+            vt = torch.from_numpy(v[b, :L, h // G]).view(1, 1, L, D)
+            ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, scale=0.45)
+            np.testing.assert_allclose(o[b, h], ref.view(D).numpy(), atol=1e-13)
+            want = torch.logsumexp(0.45 * (kt.view(L, D) @ qt.view(D)), 0).item()
+            assert abs(lse[b, h] - want) < 1e-12
+
+
+def test_decode_closed_forms():
+    B, Hq, Hkv, Lmax, D = 4, 4, 2, 17, 4
+    q, k, v = _decode_problem(B, Hq, Hkv, Lmax, D, 80)
+    lens = np.array([17, 5, 1, 0], dtype=np.int32)
+    o, _ = oracle.decode(q, k, np.ones_like(v), lens, 0.3)          # V = ones
+    np.testing.assert_allclose(o[:3], 1.0, atol=1e-13)
+    assert (o[3] == 0).all()
+    kk = np.repeat(k[:, :1], Lmax, axis=1)                              # identical keys
+    o, lse = oracle.decode(q, kk, v, lens, 0.3)
+    for b in range(3):
+        L = lens[b]
+        for h in range(Hq):
+            g = h // 2
+            np.testing.assert_allclose(o[b, h], v[b, :L, g].mean(0), atol=1e-13)
+            assert abs(lse[b, h] - (0.3 * q[b, h] @ kk[b, 0, g] + math.log(L))) < 1e-12
+    o, lse = oracle.decode(q, k, v, lens, 0.3)                          # one key, no key
+    for h in range(Hq):
+        np.testing.assert_allclose(o[2, h], v[2, 0, h // 2], atol=1e-14)
+        assert abs(lse[2, h] - 0.3 * q[2, h] @ k[2, 0, h // 2]) < 1e-13
+    assert (o[3] == 0).all() and np.isneginf(lse[3]).all()
+
+
+def test_decode_gqa_and_ignores_entries_past_the_length():
+    B, Hq, Hkv, Lmax, D = 2, 6, 2, 11, 4
+    q, k, v = _decode_problem(B, Hq, Hkv, Lmax, D, 90)
+    lens = np.array([7, 11], dtype=np.int32)
+    o1, l1 = oracle.decode(q, k, v, lens, 0.5)
+    o2, l2 = oracle.decode(q, np.repeat(k, 3, axis=2), np.repeat(v, 3, axis=2), lens, 0.5)
+    np.testing.assert_allclose(o1, o2, atol=1e-14)
+    np.testing.assert_allclose(l1, l2, atol=1e-14)
+    k2, v2 = k.copy(), v.copy()
+    k2[0, 7:], v2[0, 7:] = 1e30, np.nan
+    o3, l3 = oracle.decode(q, k2, v2, lens, 0.5)
+    assert np.array_equal(o1, o3) and np.array_equal(l1, l3)
