@@ -15,7 +15,8 @@ On one GPU the line also carries "ring": the exact merge kernel of Ring attentio
 (attn_merge, HBM-bound, against the measured copy bandwidth) and the forward of a
 4-rank ring run rank after rank on this GPU; and "ulysses": the relayout kernel around
 the Ulysses all-to-alls (HBM-bound) and forward + backward of a 4-rank Ulysses group run
-rank after rank on this GPU.  All are measured after the timed steps.
+rank after rank on this GPU; and "decode": attention of one new token per sequence over
+a 32K-token KV cache (HBM-bound).  All are measured after the timed steps.
 
 --impl reference times the fp64 CPU oracle (the reference arm of this build) on a
 bounded sample of the same workload: the first tokens of the causal sequence form
@@ -346,6 +347,49 @@ def ulysses_measurements(wr: I.Workload, q, k, v, do, stream, peaks, world=4, re
     }
 
 
+def decode_measurements(dev, stream, peaks, reps=20):
+    """Measures decode attention over a KV cache (attn_decode: split-KV kernel + merge) on
+    the two decode workloads, outside the timed step.  HBM-bound: achieved = the cached
+    K/V bytes read plus q read and o/lse written, / median CUDA-event time, against the
+    measured copy bandwidth.  The cache (1.4 GB at 16 x 32K) exceeds L2, and a 256 MB buffer
+    is written between launches so the single-sequence case (67 MB) starts cold too.
+    Values are seeded normals drawn on the GPU (their values do not change the timing)."""
+    import torch
+    from long_context_attention_fwd_b200 import ops
+
+    out = {}
+    gen = torch.Generator(device=dev).manual_seed(20261212)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    hbm = float(peaks.get("hbm_gbs"))
+    for w in I.decode_workloads()[1:]:
+        q = torch.randn((w.B, w.Hq, w.D), generator=gen, device=dev).mul_(w.qkv_mult).bfloat16()
+        k = torch.randn((w.B, w.Lmax, w.Hkv, w.D), generator=gen, device=dev).mul_(w.qkv_mult).bfloat16()
+        v = torch.randn((w.B, w.Lmax, w.Hkv, w.D), generator=gen, device=dev).mul_(w.qkv_mult).bfloat16()
+        cl = torch.tensor(w.lens, dtype=torch.int32, device=dev)
+        ws = torch.empty(ops.attn_decode_workspace_size(q, k), dtype=torch.uint8, device=dev)
+        o, lse = torch.empty_like(q), torch.empty((w.B, w.Hq), device=dev)
+        for _ in range(3):
+            ops.attn_decode(q, k, v, cl, scale=w.softmax_scale, out=o, lse=lse, workspace=ws)
+        ts = []
+        for _ in range(reps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            ops.attn_decode(q, k, v, cl, scale=w.softmax_scale, out=o, lse=lse, workspace=ws)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        ms = statistics.median(ts)
+        gbs = w.io_bytes() / (ms * 1e-3) / 1e9
+        out[w.name] = {"kernels": "attn_decode_kernel + attn_merge_kernel (strided)",
+                       "bound": "hbm", "ms": ms, "bytes": w.io_bytes(), "achieved": gbs,
+                       "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                       "tokens_per_s": w.B / (ms * 1e-3),
+                       "cache_lengths": f"{min(w.lens)}..{max(w.lens)} (sum {sum(w.lens)})"}
+        del q, k, v, ws
+    return out
+
+
 def run_gpu(args, w: I.Workload):
     import torch
     from long_context_attention_fwd_b200 import ops
@@ -476,6 +520,9 @@ def run_gpu(args, w: I.Workload):
     if (ws == 1 and dense and wr.S % 4 == 0 and wr.Hq % 4 == 0 and wr.Hkv % 4 == 0
             and not args.no_ulysses):
         uly_rows = ulysses_measurements(wr, q, k, v, do, stream, peaks)
+    dec_rows = None
+    if ws == 1 and not args.no_decode:
+        dec_rows = decode_measurements(dev, stream, peaks)
 
     if rank == 0:
         line = {
@@ -510,6 +557,8 @@ def run_gpu(args, w: I.Workload):
             line["ring"] = ring_rows
         if uly_rows is not None:
             line["ulysses"] = uly_rows
+        if dec_rows is not None:
+            line["decode"] = dec_rows
         if ws == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(wr)
         print(json.dumps(line), flush=True)
@@ -528,6 +577,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", action="store_true",
+                    help="skip the decode-attention measurements")
     ap.add_argument("--no-ulysses", action="store_true",
                     help="skip the Ulysses measurements (relayout kernel, 1-GPU Ulysses step)")
     ap.add_argument("--no-ring", action="store_true",

@@ -110,6 +110,33 @@ attn_status attn_bwd_noalloc(const void* q, const void* k, const void* v, const 
                              int B, int Hq, int Hkv, int S, int D, int causal, float scale,
                              const int32_t* cu_seqlens, void* stream);
 
+/* Bytes of device workspace attn_decode needs (0 for invalid sizes).  It holds the
+ * per-split partial results: 2 * nsplit partials of B*Hq rows (bf16 o and fp32 lse), where
+ * nsplit is fixed by (B, Hkv, Lmax). */
+size_t attn_decode_workspace_size(int B, int Hq, int Hkv, int Lmax, int D);
+
+/* Decode attention over a key/value cache: one new query token per sequence attends to
+ * all cache_len[b] cached keys of its sequence (page "ms-swift长文本训练秘诀：Ulysses并行技术
+ * 解析", section 5: serving the fine-tuned model with a 32K-token context; the arithmetic
+ * is the standard attention of page "ms-swift集成FlashAttention 2/3，长文本训练更高效",
+ * section "为什么传统注意力这么'吃'显存", one query row against the cache).
+ *     o[b][h] = sum_j softmax_j(scale * q[b][h] . k[b][j][g]) v[b][j][g],  g = h / (Hq/Hkv)
+ *     lse[b][h] = ln sum_j exp(scale * q[b][h] . k[b][j][g])
+ *   - q, o: bf16 [B][Hq][D]; k_cache, v_cache: bf16 [B][Lmax][Hkv][D]; lse: fp32 [B][Hq];
+ *     cache_len: DEVICE int32 [B], each clamped to [0, Lmax].  Cache rows at or past
+ *     cache_len[b] are never used, whatever they hold.  cache_len[b] = 0 gives o = 0 and
+ *     lse = -inf.
+ *   - The cache is split along the keys; every split writes a partial (o, lse) into
+ *     `workspace` (>= attn_decode_workspace_size bytes, 256-byte aligned, caller-owned,
+ *     no initialisation needed) and attn_merge's kernel combines them exactly.
+ *   - D in {64, 128}; Hq a multiple of Hkv with Hq/Hkv <= 128; B*Lmax and B*Hq < 2^31.
+ *   - Pointers as in every entry point (16-byte aligned tensors, 4-byte lse/cache_len).
+ *   - Deterministic. */
+attn_status attn_decode(const void* q, const void* k_cache, const void* v_cache,
+                        const int32_t* cache_len, void* o, float* lse, int B, int Hq, int Hkv,
+                        int Lmax, int D, float scale, void* workspace, size_t workspace_bytes,
+                        void* stream);
+
 /* Largest number of partial results one attn_merge call combines. */
 #define ATTN_MERGE_MAX_PARTS 16
 

@@ -56,6 +56,9 @@ _SIGNATURES = {
     "attn_selftest_umma": (_i, [_i, _i, _vp, _vp, _fp, _vp, _fp, _vp]),
     "attn_version": (_i, []),
     "attn_last_error": (ctypes.c_char_p, []),
+    "attn_decode_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
+    "attn_decode": (_i, [_vp, _vp, _vp, _vp, _vp, _fp, _i, _i, _i, _i, _i, ctypes.c_float, _vp,
+                         _sz, _vp]),
     "attn_transpose_blocks": (_i, [_vp, _vp, ctypes.c_longlong, ctypes.c_longlong,
                                    ctypes.c_longlong, _vp]),
     "attn_merge": (_i, [_vp, _vp, _i, _vp, _fp, _i, _i, _i, _i, _vp]),
@@ -136,6 +139,16 @@ def attn_merge(o_parts, lse_parts, o, lse, B, H, S, D, stream) -> int:
     la = (ctypes.c_void_p * max(n, 1))(*lse_parts)
     return lib().attn_merge(ctypes.cast(oa, _vp), ctypes.cast(la, _vp), n, o, lse, B, H, S, D,
                             stream)
+
+
+def attn_decode_workspace_size(B, Hq, Hkv, Lmax, D) -> int:
+    return lib().attn_decode_workspace_size(B, Hq, Hkv, Lmax, D)
+
+
+def attn_decode(q, k_cache, v_cache, cache_len, o, lse, B, Hq, Hkv, Lmax, D, scale, workspace,
+                workspace_bytes, stream) -> int:
+    return lib().attn_decode(q, k_cache, v_cache, cache_len, o, lse, B, Hq, Hkv, Lmax, D,
+                             float(scale), workspace, workspace_bytes, stream)
 
 
 def attn_transpose_blocks(inp, out, n_outer, n_inner, block_bytes, stream) -> int:

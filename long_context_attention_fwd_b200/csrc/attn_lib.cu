@@ -13,6 +13,7 @@
 
 #include "../../include/attn.h"
 #include "attn_bwd.cuh"
+#include "attn_decode.cuh"
 #include "attn_fwd.cuh"
 #include "attn_merge.cuh"
 #include "attn_relayout.cuh"
@@ -21,6 +22,7 @@
 using namespace attn_sm100;
 
 static_assert(merge::kMaxParts == ATTN_MERGE_MAX_PARTS, "merge part limit out of sync");
+static_assert(decode::kRegsLaunch == fwd::kRegsLaunch, "register split of the decode kernel");
 
 // Sticky device status: [0] status bits, [1] site code of the first timeout.
 static __device__ unsigned g_attn_status[2];
@@ -106,19 +108,23 @@ attn_status device_setup(DeviceState** out, const void* ptr = nullptr) {
       e = e ? e : cudaFuncSetAttribute(fwd::attn_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, fwd::Cfg<128>::SMEM_ALLOC);
       e = e ? e : cudaFuncSetAttribute(bwd::attn_bwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, bwd::Cfg<64>::SMEM_ALLOC);
       e = e ? e : cudaFuncSetAttribute(bwd::attn_bwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, bwd::Cfg<128>::SMEM_ALLOC);
+      e = e ? e : cudaFuncSetAttribute(decode::attn_decode_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, decode::Cfg<64>::SMEM_ALLOC);
+      e = e ? e : cudaFuncSetAttribute(decode::attn_decode_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, decode::Cfg<128>::SMEM_ALLOC);
       e = e ? e : cudaFuncSetAttribute(selftest::umma_selftest_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, 32768 + 128 * 64 * 2 + 2048);
       e = e ? e : cudaFuncSetAttribute(selftest::umma_selftest_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, 32768 + 128 * 128 * 2 + 2048);
       if (e != cudaSuccess) return fail_cuda("cudaFuncSetAttribute", e);
       // The kernels re-split registers between warpgroups with setmaxnreg; that is only
       // safe when each thread starts with exactly the budget the split was sized for.
-      const void* split_kernels[4] = {
+      const void* split_kernels[6] = {
           reinterpret_cast<const void*>(fwd::attn_fwd_kernel<64>),
           reinterpret_cast<const void*>(fwd::attn_fwd_kernel<128>),
           reinterpret_cast<const void*>(bwd::attn_bwd_kernel<64>),
-          reinterpret_cast<const void*>(bwd::attn_bwd_kernel<128>)};
-      const int split_regs[4] = {fwd::kRegsLaunch, fwd::kRegsLaunch, bwd::kRegsLaunch,
-                                 bwd::kRegsLaunch};
-      for (int i = 0; i < 4; ++i) {
+          reinterpret_cast<const void*>(bwd::attn_bwd_kernel<128>),
+          reinterpret_cast<const void*>(decode::attn_decode_kernel<64>),
+          reinterpret_cast<const void*>(decode::attn_decode_kernel<128>)};
+      const int split_regs[6] = {fwd::kRegsLaunch, fwd::kRegsLaunch, bwd::kRegsLaunch,
+                                 bwd::kRegsLaunch, decode::kRegsLaunch, decode::kRegsLaunch};
+      for (int i = 0; i < 6; ++i) {
         cudaFuncAttributes fa;
         if ((e = cudaFuncGetAttributes(&fa, split_kernels[i])) != cudaSuccess)
           return fail_cuda("cudaFuncGetAttributes", e);
@@ -203,6 +209,51 @@ WsLayout ws_layout(int B, int Hq, long long T, int D) {
   w.delta = w.lse2 + round_up(size_t(Hq) * w.ntile * 128 * sizeof(float), 256);
   w.total = w.delta + round_up(size_t(Hq) * w.ntile * 128 * sizeof(float), 256);
   return w;
+}
+
+// Split plan of decode: tiles per split and splits per (sequence, kv head), a function
+// of the shapes only (so the workspace size needs no device query).  Aims at about two
+// CTAs per SM of a 148-SM B200 in total, at least four 128-key tiles per split, and at
+// most decode_max_parts() partial results.
+constexpr int kPlanSMs = 148;
+int decode_max_parts() { return merge::kMaxStridedParts; }
+void decode_plan(int B, int Hkv, int Lmax, int* nsplit, int* tps) {
+  const long long ntile = (Lmax + 127) / 128;
+  const long long units = (long long)B * Hkv;
+  long long t = (units * ntile + 2 * kPlanSMs - 1) / (2 * kPlanSMs);
+  if (t < 4) t = 4;
+  if (t > ntile) t = ntile;
+  long long ns = (ntile + t - 1) / t;
+  if (2 * ns > decode_max_parts()) {
+    ns = decode_max_parts() / 2;
+    t = (ntile + ns - 1) / ns;
+    ns = (ntile + t - 1) / t;
+  }
+  *nsplit = int(ns);
+  *tps = int(t);
+}
+struct DecodeWs {
+  size_t o_part, lse_part, total;
+  int nsplit, tps, nparts;
+};
+DecodeWs decode_ws(int B, int Hq, int Hkv, int Lmax, int D) {
+  DecodeWs w;
+  decode_plan(B, Hkv, Lmax, &w.nsplit, &w.tps);
+  w.nparts = 2 * w.nsplit;
+  const size_t rows = size_t(B) * Hq;
+  w.o_part = 0;
+  w.lse_part = round_up(size_t(w.nparts) * rows * D * 2, 256);
+  w.total = w.lse_part + round_up(size_t(w.nparts) * rows * 4, 256);
+  return w;
+}
+attn_status check_decode_sizes(int B, int Hq, int Hkv, int Lmax, int D, float scale) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || Lmax < 1) return ATTN_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0 || Hq / Hkv > 128) return ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+  if ((long long)B * Lmax >= (1ll << 31) - 256 || (long long)B * Hq >= (1ll << 31) - 256)
+    return ATTN_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+  return ATTN_OK;
 }
 
 }  // namespace
@@ -371,6 +422,9 @@ attn_status attn_merge(const void* const* o_parts, const float* const* lse_parts
     p.o_parts[j] = nullptr;
     p.lse_parts[j] = nullptr;
   }
+  p.o_base = nullptr;
+  p.lse_base = nullptr;
+  p.o_stride = p.lse_stride = 0;
   if (!aligned(o, 16) || !aligned(lse, 4)) return ATTN_ERR_MISALIGNED;
   DeviceState* dev = nullptr;
   attn_status st = device_setup(&dev, o);
@@ -399,6 +453,89 @@ attn_status attn_merge(const void* const* o_parts, const float* const* lse_parts
     else merge::attn_merge_kernel<128, 4, 1><<<grid, thr, 0, s>>>(p);
   }
   return check_launch("attn_merge_kernel launch");
+}
+
+size_t attn_decode_workspace_size(int B, int Hq, int Hkv, int Lmax, int D) {
+  if (check_decode_sizes(B, Hq, Hkv, Lmax, D, 1.f) != ATTN_OK) return 0;
+  return decode_ws(B, Hq, Hkv, Lmax, D).total;
+}
+
+attn_status attn_decode(const void* q, const void* k_cache, const void* v_cache,
+                        const int32_t* cache_len, void* o, float* lse, int B, int Hq, int Hkv,
+                        int Lmax, int D, float scale, void* workspace, size_t workspace_bytes,
+                        void* stream) {
+  attn_status st = check_decode_sizes(B, Hq, Hkv, Lmax, D, scale);
+  if (st != ATTN_OK) return st;
+  if (!q || !k_cache || !v_cache || !cache_len || !o || !lse || !workspace)
+    return ATTN_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(o, 16) ||
+      !aligned(workspace, 256) || !aligned(lse, 4) || !aligned(cache_len, 4))
+    return ATTN_ERR_MISALIGNED;
+  const DecodeWs w = decode_ws(B, Hq, Hkv, Lmax, D);
+  if (workspace_bytes < w.total) return ATTN_ERR_INVALID_ARG;
+  DeviceState* dev = nullptr;
+  if ((st = device_setup(&dev, q)) != ATTN_OK) return st;
+
+  CUtensorMap mq, mk, mv;
+  if (make_map(&mq, q, D, 1, (long long)B * Hq) || make_map(&mk, k_cache, D, Hkv, (long long)B * Lmax) ||
+      make_map(&mv, v_cache, D, Hkv, (long long)B * Lmax))
+    return ATTN_ERR_CUDA;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  decode::Params p;
+  p.cache_len = cache_len;
+  p.o_part = reinterpret_cast<__nv_bfloat16*>(ws + w.o_part);
+  p.lse_part = reinterpret_cast<float*>(ws + w.lse_part);
+  p.Hq = Hq;
+  p.G = Hq / Hkv;
+  p.Hkv = Hkv;
+  p.Lmax = Lmax;
+  p.nsplit = w.nsplit;
+  p.tps = w.tps;
+  p.rows = B * Hq;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.status = dev->status;
+  p.timeout_ns = g_timeout_ns.load();
+  const long long nblocks = (long long)B * Hkv * w.nsplit;
+  if (nblocks >= (1ll << 31)) return ATTN_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (D == 64)
+    decode::attn_decode_kernel<64><<<unsigned(nblocks), decode::kThreads, decode::Cfg<64>::SMEM_ALLOC, s>>>(mq, mk, mv, p);
+  else
+    decode::attn_decode_kernel<128><<<unsigned(nblocks), decode::kThreads, decode::Cfg<128>::SMEM_ALLOC, s>>>(mq, mk, mv, p);
+  if ((st = check_launch("attn_decode_kernel launch")) != ATTN_OK) return st;
+
+  // Combine the 2 * nsplit partials of every (sequence, head) row exactly.
+  merge::Params mp;
+  for (int j = 0; j < merge::kMaxParts; ++j) {
+    mp.o_parts[j] = nullptr;
+    mp.lse_parts[j] = nullptr;
+  }
+  const unsigned rows = unsigned(B) * unsigned(Hq);
+  mp.o_base = reinterpret_cast<const uint4*>(ws + w.o_part);
+  mp.lse_base = reinterpret_cast<const float*>(ws + w.lse_part);
+  mp.o_stride = size_t(rows) * D * 2 / 16;
+  mp.lse_stride = rows;
+  mp.o = static_cast<uint4*>(o);
+  mp.lse = lse;
+  mp.nparts = w.nparts;
+  mp.H = 1;
+  mp.S = rows;
+  mp.rows = rows;
+  const int var = merge::variant_for(w.nparts);
+  const unsigned rows_per_block =
+      unsigned(merge::kThreads / (D / 8)) * unsigned(merge::kVariantRows[var]);
+  const unsigned need = (rows + rows_per_block - 1) / rows_per_block;
+  const unsigned wave = dev->merge_grid[D == 64 ? 0 : 1][var];
+  const dim3 grid(need < wave ? need : wave);
+  const unsigned thr = merge::kThreads;
+  if (D == 64) {
+    if (var == 1) merge::attn_merge_kernel<64, 2, 2><<<grid, thr, 0, s>>>(mp);
+    else merge::attn_merge_kernel<64, 4, 1><<<grid, thr, 0, s>>>(mp);
+  } else {
+    if (var == 1) merge::attn_merge_kernel<128, 2, 2><<<grid, thr, 0, s>>>(mp);
+    else merge::attn_merge_kernel<128, 4, 1><<<grid, thr, 0, s>>>(mp);
+  }
+  return check_launch("attn_merge_kernel launch (decode)");
 }
 
 attn_status attn_transpose_blocks(const void* in, void* out, long long n_outer, long long n_inner,

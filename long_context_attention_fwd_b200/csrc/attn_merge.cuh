@@ -31,15 +31,30 @@ namespace merge {
 constexpr int kMaxParts = 16;
 constexpr int kThreads = 256;
 
+constexpr int kMaxStridedParts = 256;
+
 struct Params {
   const uint4* o_parts[kMaxParts];    // [T][H][D] bf16 as groups of eight
   const float* lse_parts[kMaxParts];  // [B][H][S] fp32 (lse layout of the forward)
+  // Strided form (o_base != nullptr): partial j is o_base + j * o_stride and
+  // lse_base + j * lse_stride; used for the many per-split partials of decode.
+  const uint4* o_base;
+  const float* lse_base;
+  size_t o_stride;                    // in 16-byte units
+  size_t lse_stride;                  // in floats
   uint4* o;                           // [T][H][D] bf16
   float* lse;                         // [B][H][S]
   int nparts;
   unsigned H, S;                      // T = B * S tokens
   unsigned rows;                      // T * H  (< 2^31, checked on the host)
 };
+
+__device__ __forceinline__ const uint4* part_o(const Params& p, int j) {
+  return p.o_base ? p.o_base + size_t(j) * p.o_stride : p.o_parts[j];
+}
+__device__ __forceinline__ const float* part_lse(const Params& p, int j) {
+  return p.lse_base ? p.lse_base + size_t(j) * p.lse_stride : p.lse_parts[j];
+}
 
 __device__ __forceinline__ void acc_bf16x8(float (&acc)[8], const uint4 x, const float w) {
   const uint32_t u[4] = {x.x, x.y, x.z, x.w};
@@ -62,13 +77,13 @@ __device__ __forceinline__ void merge_row(const Params& p, const float (&l)[NP],
 #pragma unroll
   for (int u = 0; u < NP; ++u) m = fmaxf(m, l[u]);
   if (kMore)
-    for (int j = NP; j < p.nparts; ++j) m = fmaxf(m, p.lse_parts[j][li]);
+    for (int j = NP; j < p.nparts; ++j) m = fmaxf(m, part_lse(p, j)[li]);
   if (m == -INFINITY) return;  // nothing visible: o = 0, lse = -inf
   float s = 0.f;
 #pragma unroll
   for (int u = 0; u < NP; ++u) s += expf(l[u] - m);  // exp(-inf) = 0 for absent partials
   if (kMore)
-    for (int j = NP; j < p.nparts; ++j) s += expf(p.lse_parts[j][li] - m);
+    for (int j = NP; j < p.nparts; ++j) s += expf(part_lse(p, j)[li] - m);
   const float inv = 1.f / s;
   lse_out = m + logf(s);
 #pragma unroll
@@ -78,10 +93,10 @@ __device__ __forceinline__ void merge_row(const Params& p, const float (&l)[NP],
     for (int j0 = NP; j0 < p.nparts; j0 += NP) {
 #pragma unroll
       for (int u = 0; u < NP; ++u)
-        if (j0 + u < p.nparts) x[u] = __ldcs(p.o_parts[j0 + u] + off);
+        if (j0 + u < p.nparts) x[u] = __ldcs(part_o(p, j0 + u) + off);
 #pragma unroll
       for (int u = 0; u < NP; ++u)
-        if (j0 + u < p.nparts) acc_bf16x8(acc, x[u], expf(p.lse_parts[j0 + u][li] - m) * inv);
+        if (j0 + u < p.nparts) acc_bf16x8(acc, x[u], expf(part_lse(p, j0 + u)[li] - m) * inv);
     }
 }
 
@@ -120,8 +135,8 @@ __global__ void __launch_bounds__(kThreads) attn_merge_kernel(const __grid_const
 #pragma unroll
         for (int u = 0; u < NP; ++u)
           if (u < p.nparts) {
-            l[k][u] = p.lse_parts[u][li[k]];
-            x[k][u] = __ldcs(p.o_parts[u] + off[k]);
+            l[k][u] = part_lse(p, u)[li[k]];
+            x[k][u] = __ldcs(part_o(p, u) + off[k]);
           }
       }
     }

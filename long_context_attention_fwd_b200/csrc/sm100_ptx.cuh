@@ -106,6 +106,17 @@ __device__ __forceinline__ unsigned long long drain_ns(volatile int* abort_flag,
   return *abort_flag ? 20000000ull : timeout_ns;
 }
 
+// Drain wait that reports failure: a drain that does not finish means the kernel's own
+// accounting of in-flight operations is wrong.  The kernel still exits; the status word
+// records a timeout at `site`, so the host sees it.
+__device__ __forceinline__ bool mbar_drain_checked(uint64_t* bar, uint32_t parity,
+                                                   const WaitCtl& w, unsigned site) {
+  if (mbar_drain(bar, parity, drain_ns(w.abort, w.timeout_ns))) return true;
+  atomicOr(w.status, kStatusTimeout);
+  atomicCAS(w.status + 1, 0u, site);
+  return false;
+}
+
 // ------------------------------------------------------------------ TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(m) : "memory");

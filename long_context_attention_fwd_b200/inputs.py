@@ -39,6 +39,7 @@ _M2 = np.uint64(0x94D049BB133111EB)
 
 # Stream tags: one per tensor kind.
 TAG_Q, TAG_K, TAG_V, TAG_DO, TAG_LEN, TAG_OUT_Q, TAG_OUT_K = 1, 2, 3, 4, 5, 6, 7
+TAG_CACHE_LEN = 8
 
 _CHUNK = 1 << 22
 
@@ -261,3 +262,78 @@ def flop_fwd(w: Workload) -> float:
 def flop_bwd(w: Workload) -> float:
     """Backward FLOP convention: 2.5x the forward count."""
     return 2.5 * flop_fwd(w)
+
+
+# ---------------------------------------------------------------- decode over a KV cache
+@dataclass
+class DecodeWorkload:
+    """One decode step: a new query token per sequence against its key/value cache.
+    q [B,Hq,D]; k/v cache [B,Lmax,Hkv,D]; cache_len [B] (entries past it are not used)."""
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    Lmax: int
+    D: int
+    lens: List[int]
+    qkv_mult: float = 0.5
+    seed: int = 20261202
+    scale: Optional[float] = None
+
+    @property
+    def softmax_scale(self) -> float:
+        return self.scale if self.scale is not None else 1.0 / math.sqrt(self.D)
+
+    def cache_bytes(self) -> int:
+        """Bytes of K and V the step must read: sum of lengths x Hkv x D x 2 bytes x 2."""
+        return int(sum(self.lens)) * self.Hkv * self.D * 2 * 2
+
+    def io_bytes(self) -> int:
+        """Algorithmic bytes of one step: the cache read, q read, o and lse written."""
+        return self.cache_bytes() + self.B * self.Hq * (self.D * 2 * 2 + 4)
+
+
+def decode_lengths(seed: int, B: int, lo: int, hi: int) -> List[int]:
+    """B cache lengths uniform on [lo, hi] (inclusive)."""
+    u = uniform(stream_key(seed, TAG_CACHE_LEN), B)
+    return [lo + int(math.floor(x * (hi - lo + 1))) for x in u]
+
+
+def make_decode_inputs(w: DecodeWorkload, poison_tail: bool = True) -> dict:
+    """bf16 bit tensors q [B,Hq,D], k/v [B,Lmax,Hkv,D] and cache_len int32 [B].  With
+    poison_tail, cache entries past each length hold bf16 NaN, so that any read of them
+    shows up in the output."""
+    s = w.seed
+    q = normal_bf16(stream_key(s, TAG_Q), (w.B, w.Hq, w.D), w.qkv_mult)
+    k = normal_bf16(stream_key(s, TAG_K), (w.B, w.Lmax, w.Hkv, w.D), w.qkv_mult)
+    v = normal_bf16(stream_key(s, TAG_V), (w.B, w.Lmax, w.Hkv, w.D), w.qkv_mult)
+    if poison_tail:
+        for b, L in enumerate(w.lens):
+            k[b, L:] = 0x7FC0
+            v[b, L:] = 0x7FC0
+    return {"q": q, "k": k, "v": v, "cache_len": np.asarray(w.lens, dtype=np.int32)}
+
+
+def decode_workloads() -> List[DecodeWorkload]:
+    """Decode steps at the pages' 32K deployment context with Qwen2.5-7B attention shapes,
+    and a small case whose lengths sit on and around the 128-key tile edges."""
+    return [
+        DecodeWorkload("decode_edges_B8_gqa8x2_D64", B=8, Hq=8, Hkv=2, Lmax=700, D=64,
+                       lens=[0, 1, 127, 128, 129, 255, 700, 513], qkv_mult=1.0,
+                       seed=20261202 + 10),
+        DecodeWorkload("qwen2.5-7b_decode_B1_L32768", B=1, Hq=28, Hkv=4, Lmax=32768, D=128,
+                       lens=[32768], seed=20261202 + 11),
+        DecodeWorkload("qwen2.5-7b_decode_B16_L16K-32K", B=16, Hq=28, Hkv=4, Lmax=32768, D=128,
+                       lens=decode_lengths(20261202 + 12, 16, 16384, 32768),
+                       seed=20261202 + 12),
+    ]
+
+
+def decode_workload(name_or_index) -> DecodeWorkload:
+    ws = decode_workloads()
+    if isinstance(name_or_index, int):
+        return ws[name_or_index]
+    for w in ws:
+        if w.name == name_or_index:
+            return w
+    raise KeyError(name_or_index)

@@ -5,6 +5,7 @@
     dq, dk, dv = attn_bwd(q, k, v, o, lse, do, causal=True)
     o = attention(q, k, v, causal=True)                        # autograd-aware
     o, lse = attn_merge([o1, o2], [lse1, lse2])                # exact merge of key-chunk partials
+    o, lse = attn_decode(q, k_cache, v_cache, cache_len)       # one new token per sequence
 
 All arithmetic runs in libattn.so; these functions only check shapes, allocate
 outputs with torch and pass raw pointers and the current CUDA stream.
@@ -191,3 +192,38 @@ def transpose_blocks(x: torch.Tensor, n_outer: int, n_inner: int,
                                     blk * x.element_size(), _stream(x.device))
     capi.check(st, "attn_transpose_blocks")
     return out
+
+
+def attn_decode_workspace_size(q: torch.Tensor, k_cache: torch.Tensor) -> int:
+    B, Hq, D = q.shape
+    _, Lmax, Hkv, _ = k_cache.shape
+    return capi.attn_decode_workspace_size(B, Hq, Hkv, Lmax, D)
+
+
+def attn_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                cache_len: torch.Tensor, scale: Optional[float] = None,
+                out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                workspace: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Decode attention: q [B,Hq,D] against k/v cache [B,Lmax,Hkv,D] with cache_len int32
+    [B] (on the GPU).  Returns (o [B,Hq,D] bf16, lse [B,Hq] fp32)."""
+    _check_inputs(q, k_cache, v_cache)
+    if q.dim() != 3 or k_cache.dim() != 4 or v_cache.shape != k_cache.shape:
+        raise ValueError("q must be [B,Hq,D] and the caches [B,Lmax,Hkv,D]")
+    B, Hq, D = q.shape
+    Bk, Lmax, Hkv, Dk = k_cache.shape
+    if Bk != B or Dk != D:
+        raise ValueError("cache shape does not match q")
+    if cache_len.dtype != torch.int32 or not cache_len.is_cuda or cache_len.numel() != B:
+        raise ValueError("cache_len must be an int32 CUDA tensor of B entries")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device) if lse is None else lse
+    need = capi.attn_decode_workspace_size(B, Hq, Hkv, Lmax, D)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    st = capi.attn_decode(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+                          cache_len.data_ptr(), out.data_ptr(), lse.data_ptr(), B, Hq, Hkv, Lmax,
+                          D, scale, workspace.data_ptr(), workspace.numel(), _stream(q.device))
+    capi.check(st, "attn_decode")
+    return out, lse

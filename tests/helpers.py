@@ -105,6 +105,9 @@ class GpuRun:
                                                  causal=w.causal, scale=w.softmax_scale,
                                                  cu_seqlens=self.cu, dq=dq, dk=dk, dv=dv)
         torch.cuda.synchronize()
+        from long_context_attention_fwd_b200 import capi
+        st, site = capi.attn_device_status(None)   # no device wait may have run out
+        assert st == capi.ATTN_OK, (capi.strerror(st), hex(site))
 
     def np_out(self):
         """GPU results as fp64 numpy in the oracle's layouts ([T,H,D], lse [B,Hq,S] or [Hq,T])."""

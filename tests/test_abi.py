@@ -106,3 +106,22 @@ def test_transpose_blocks_validation():
     assert t(A + 8, A + (1 << 20), 2, 2, 16, None) == capi.ATTN_ERR_MISALIGNED
     assert t(A, A + 32, 2, 2, 16, None) == capi.ATTN_ERR_INVALID_ARG             # overlap
     assert t(A, A + (1 << 40), 1 << 20, 1 << 8, 1 << 10, None) == capi.ATTN_ERR_INVALID_ARG
+
+
+def test_decode_validation_and_workspace():
+    ws = capi.attn_decode_workspace_size(16, 28, 4, 32768, 128)
+    assert ws > 0
+    assert capi.attn_decode_workspace_size(0, 28, 4, 32768, 128) == 0
+    assert capi.attn_decode_workspace_size(1, 28, 3, 1024, 128) == 0      # Hq % Hkv
+    assert capi.attn_decode_workspace_size(1, 256, 1, 1024, 128) == 0     # Hq/Hkv > 128
+    assert capi.attn_decode_workspace_size(1, 28, 4, 1024, 96) == 0
+    d = capi.attn_decode
+    need = capi.attn_decode_workspace_size(2, 8, 2, 512, 64)
+    args = (A, A, A, A, A, A, 2, 8, 2, 512, 64, 0.125)
+    assert d(*args, A, need - 1, None) == capi.ATTN_ERR_INVALID_ARG
+    assert d(*args, None, need, None) == capi.ATTN_ERR_INVALID_ARG
+    assert d(*args, A + 16, need, None) == capi.ATTN_ERR_MISALIGNED      # workspace 256-aligned
+    assert d(A + 8, *args[1:], A, need, None) == capi.ATTN_ERR_MISALIGNED
+    assert d(A, A, A, A + 2, A, A, 2, 8, 2, 512, 64, 0.125, A, need, None) == capi.ATTN_ERR_MISALIGNED
+    assert d(A, A, A, A, A, A, 2, 8, 2, 512, 96, 0.125, A, need, None) == capi.ATTN_ERR_UNSUPPORTED
+    assert d(A, A, A, A, A, A, 2, 8, 2, 512, 64, float("nan"), A, need, None) == capi.ATTN_ERR_INVALID_ARG

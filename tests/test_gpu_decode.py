@@ -1,0 +1,91 @@
+"""Decode attention over a key/value cache (attn_decode) on the GPU against the fp64
+oracle, element by element: every output row of every workload.
+
+The caches hold bf16 NaN past each sequence's length, so a read of any entry past the
+length would show up as NaN in the output.  Cases cover lengths on and around the
+128-key tile edges (0, 1, 127, 128, 129, ...), grouped-query ratios 1, 7 and 64 (the
+last needs two warps of rows per stream), both head dimensions, the split plans of a
+single 32K sequence (64 splits) and of 16 sequences of 16K-32K keys, and determinism.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from helpers import TOL_LSE, bits_of, f64, o_error_report, torch_bf16
+from long_context_attention_fwd_b200 import inputs as I
+
+torch = pytest.importorskip("torch")
+
+
+def _run(w):
+    from long_context_attention_fwd_b200 import ops
+    x = I.make_decode_inputs(w, poison_tail=True)
+    q = torch_bf16(x["q"]).view(w.B, w.Hq, w.D)
+    k = torch_bf16(x["k"]).view(w.B, w.Lmax, w.Hkv, w.D)
+    v = torch_bf16(x["v"]).view(w.B, w.Lmax, w.Hkv, w.D)
+    cl = torch.from_numpy(x["cache_len"]).cuda()
+    o = torch.empty_like(q)
+    o.view(torch.int16).fill_(0x7FC0)
+    lse = torch.full((w.B, w.Hq), float("nan"), device="cuda")
+    o, lse = ops.attn_decode(q, k, v, cl, scale=w.softmax_scale, out=o, lse=lse)
+    torch.cuda.synchronize()
+    from long_context_attention_fwd_b200 import capi
+    st, site = capi.attn_device_status(None)   # no wait or drain may have run out
+    assert st == capi.ATTN_OK, (capi.strerror(st), hex(site))
+    return x, o, lse
+
+
+def _check(w, x, o, lse):
+    # oracle on the same bits, with the poisoned tail replaced by zeros (never read)
+    kf, vf = f64(x["k"]).copy(), f64(x["v"]).copy()
+    for b, L in enumerate(w.lens):
+        kf[b, L:] = 0.0
+        vf[b, L:] = 0.0
+    qf = f64(x["q"])
+    o_r, l_r = oracle.decode(qf, kf, vf, x["cache_len"], w.softmax_scale)
+    oa_r, _ = oracle.decode(qf, kf, np.abs(vf), x["cache_len"], w.softmax_scale)
+    og = f64(bits_of(o)).reshape(w.B, w.Hq, w.D)
+    lg = lse.double().cpu().numpy()
+    empty = np.array(w.lens) == 0
+    assert not np.isnan(og).any() and not np.isnan(lg).any()
+    assert (og[empty] == 0).all() and np.isneginf(lg[empty]).all()
+    full = ~empty
+    rep = o_error_report(og[full], o_r[full], oa_r[full])
+    assert rep["n_over_model"] == 0 and rep["max_abs"] <= 1e-2, rep
+    assert np.abs(lg[full] - l_r[full]).max() <= TOL_LSE
+    return rep
+
+
+CASES = [
+    I.decode_workload(0),
+    I.DecodeWorkload("decode_gqa7_D128", B=3, Hq=28, Hkv=4, Lmax=1000, D=128,
+                     lens=[1000, 385, 129], seed=41),
+    I.DecodeWorkload("decode_mqa64_D128", B=2, Hq=64, Hkv=1, Lmax=520, D=128, lens=[520, 1],
+                     seed=42),
+    I.DecodeWorkload("decode_mha_D64", B=2, Hq=8, Hkv=8, Lmax=300, D=64, lens=[300, 0], seed=43),
+    I.DecodeWorkload("decode_one_tile_D128", B=4, Hq=28, Hkv=4, Lmax=128, D=128,
+                     lens=[128, 64, 1, 127], seed=44),
+]
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("w", CASES, ids=[c.name for c in CASES])
+def test_decode_small_matches_oracle(w):
+    x, o, lse = _run(w)
+    _check(w, x, o, lse)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("idx", [1, 2], ids=["B1_L32K", "B16_L16K-32K"])
+def test_decode_full_size_matches_oracle(idx):
+    w = I.decode_workload(idx)
+    x, o, lse = _run(w)
+    _check(w, x, o, lse)
+
+
+@pytest.mark.gpu
+def test_decode_deterministic():
+    w = CASES[1]
+    _, o1, l1 = _run(w)
+    _, o2, l2 = _run(w)
+    assert torch.equal(o1.view(torch.int16), o2.view(torch.int16)) and torch.equal(l1, l2)
