@@ -22,9 +22,11 @@
 //                   accumulator with coalesced vector reductions.  dK/dV stay deterministic.
 //   dq_convert      dq = bf16(scale * accumulator).
 //
-// Warps: 0-3 compute P^T and dS^T (one thread per key row), 4-7 drain dQ from TMEM
-// and reduce it into the accumulator, 8 is the TMA producer, 9 issues the MMAs,
-// 10-11 only complete the control warpgroup for the register split.
+// Warps: 0-3 and 4-7 compute P^T and dS^T (one thread per key row; warps 0-3 take query
+// columns 0-63 of the tile, warps 4-7 columns 64-127, which halves the per-thread chain
+// that paces the loop), 8-11 drain dQ from TMEM and reduce it into the accumulator,
+// 12 is the TMA producer, 13 issues the MMAs, 14-15 only complete the control warpgroup
+// for the register split.
 #pragma once
 #include <cuda_bf16.h>
 #include "attn_common.cuh"
@@ -33,16 +35,17 @@
 namespace attn_sm100 {
 namespace bwd {
 
-constexpr int kThreads = 384;    // 12 warps; warps 10-11 only complete the control warpgroup
-constexpr int kWarpTMA = 8;
-constexpr int kWarpMMA = 9;
-// Register split (setmaxnreg): the launch gives every thread 168 registers
-// (384 x 168 = 64512); the control warpgroup (warps 8-11) drops to 72 and the two
-// compute warpgroups rise to 216: 128 x 72 + 256 x 216 = 64512, exactly the pool.
-constexpr int kRegsLaunch = 168;
+constexpr int kThreads = 512;    // 16 warps; warps 14-15 only complete the control warpgroup
+constexpr int kWarpTMA = 12;
+constexpr int kWarpMMA = 13;
+// Register split (setmaxnreg): the launch gives every thread 128 registers
+// (512 x 128 = 65536); the control warpgroup (warps 12-15) drops to 72 and the three
+// compute warpgroups (P/dS, P/dS, dQ drain) rise to 144:
+// 128 x 72 + 384 x 144 = 64512 <= 65536 (the smallest split ptxas compiles without spills).
+constexpr int kRegsLaunch = 128;
 constexpr int kRegsControl = 72;
-constexpr int kRegsCompute = 216;
-static_assert(128 * kRegsControl + 256 * kRegsCompute <= kThreads * kRegsLaunch, "register split");
+constexpr int kRegsCompute = 144;
+static_assert(128 * kRegsControl + 384 * kRegsCompute <= kThreads * kRegsLaunch, "register split");
 constexpr int kSlab = 128 * 128;
 
 struct Params {
@@ -229,8 +232,8 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
     mbar_init(s_full, 1);
     mbar_init(dp_full, 1);
-    mbar_init(p_full, 4);
-    mbar_init(ds_full, 4);
+    mbar_init(p_full, 8);
+    mbar_init(ds_full, 8);
     mbar_init(dq_full, 1);
     mbar_init(dq_free, 4);
     mbar_init(dkv_final, 1);
@@ -253,7 +256,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   const uint32_t tmem = *tmem_slot;
   const WaitCtl wc{p.status, abort_flag, p.timeout_ns};
 
-  if (warp >= 8) {
+  if (warp >= 12) {
     reg_dealloc<kRegsControl>();
     if (warp == kWarpTMA && lane == 0) {
       // ---------------------------------------------------------- producer
@@ -268,6 +271,13 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const uint32_t ph = ((it >> 1) & 1) ^ 1;
         const int hq = g * p.G + it % p.G;
         const int m = nq - 1 - it / p.G;
+        // dO first: its stage frees at the dP MMA, earlier than Q's (freed at the dK MMA).
+        if (!mbar_wait(&do_empty[st], ph, wc, kSiteDoEmpty)) break;
+        mbar_arrive_expect_tx(&do_full[st], C::TILE);
+        for (int hf = 0; hf < D / 64; ++hf)
+          tma_load_3d(&tm_do, &do_full[st], smem + C::OFF_DO + st * C::TILE + hf * kSlab, hf * 64,
+                      hq, start + 128 * m);
+        ++ndo_issued;
         if (!mbar_wait(&q_empty[st], ph, wc, kSiteQEmpty)) break;
         mbar_arrive_expect_tx(&q_full[st], C::TILE + 1024);
         for (int hf = 0; hf < D / 64; ++hf)
@@ -277,12 +287,6 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         bulk_load(lse_s + st * 128, p.lse2 + wi, 512, &q_full[st]);
         bulk_load(delta_s + st * 128, p.delta + wi, 512, &q_full[st]);
         ++nq_issued;
-        if (!mbar_wait(&do_empty[st], ph, wc, kSiteDoEmpty)) break;
-        mbar_arrive_expect_tx(&do_full[st], C::TILE);
-        for (int hf = 0; hf < D / 64; ++hf)
-          tma_load_3d(&tm_do, &do_full[st], smem + C::OFF_DO + st * C::TILE + hf * kSlab, hf * 64,
-                      hq, start + 128 * m);
-        ++ndo_issued;
       }
       mbar_drain(kv_full, 0, drain_ns(abort_flag, p.timeout_ns));
       for (int st = 0; st < 2; ++st) {
@@ -313,22 +317,25 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         issue_T(C::COL_S, kb, smem_u32(smem + C::OFF_Q));
         mma_commit(s_full);
       }
+      // P^T and dS^T halves sit in TMEM columns [0, 32) and [96, 128) of their regions
+      // (warps 0-3 / warps 4-7, bf16 pairs): A-operand column of 16-row step kk.
+      auto a_col = [](int kk) -> uint32_t { return kk < 4 ? kk * 8 : 96 + (kk - 4) * 8; };
       for (int it = 0; it < iters && ok; ++it) {
         const int st = it & 1;
         const uint32_t ph = (it >> 1) & 1;
         const uint32_t qb = smem_u32(smem + C::OFF_Q + st * C::TILE);
         const uint32_t dob = smem_u32(smem + C::OFF_DO + st * C::TILE);
-        if (it > 0 && !(ok = mbar_wait(dq_free, (it - 1) & 1, wc, kSiteDqFree))) break;
         if (!(ok = mbar_wait(&do_full[st], ph, wc, kSiteDoFull))) break;
-        tc_fence_after();
-        issue_T(C::COL_DP, vb, dob);  // dP^T = V dO^T
-        mma_commit(dp_full);
         if (!(ok = mbar_wait(p_full, it & 1, wc, kSitePFull))) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)  // dV += P^T dO
-          mma_ts(tmem + C::COL_DV, tmem + C::COL_S + kk * 8, sdesc_sw128(dob + kk * 2048, kSlab, 1024),
+          mma_ts(tmem + C::COL_DV, tmem + C::COL_S + a_col(kk), sdesc_sw128(dob + kk * 2048, kSlab, 1024),
                  idKV, (it > 0 || kk > 0) ? 1u : 0u);
+        if (it > 0 && !(ok = mbar_wait(dq_free, (it - 1) & 1, wc, kSiteDqFree))) break;
+        tc_fence_after();
+        issue_T(C::COL_DP, vb, dob);  // dP^T = V dO^T (into the columns dQ was drained from)
+        mma_commit(dp_full);
         mma_commit(&do_empty[st]);
         if (it + 1 < iters) {
           if (!(ok = mbar_wait(&q_full[st ^ 1], ((it + 1) >> 1) & 1, wc, kSiteQFull))) break;
@@ -340,7 +347,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)  // dK += dS^T Q
-          mma_ts(tmem + C::COL_DK, tmem + C::COL_DP + kk * 8, sdesc_sw128(qb + kk * 2048, kSlab, 1024),
+          mma_ts(tmem + C::COL_DK, tmem + C::COL_DP + a_col(kk), sdesc_sw128(qb + kk * 2048, kSlab, 1024),
                  idKV, (it > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&q_empty[st]);
 #pragma unroll
@@ -353,17 +360,26 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       mma_commit(drain);
       mbar_drain(drain, 0, drain_ns(abort_flag, p.timeout_ns));
     }
-  } else if (warp < 4) {
+  } else if (warp < 8) {
     reg_alloc<kRegsCompute>();
     // ------------------------------------------------------------ P^T and dS^T
-    const int qw = warp;
+    // Warpgroup wg takes query columns cb .. cb+63 of the tile (cb = 64 wg); thread r owns
+    // key row r.  The bf16 results are stored in place, packed two per 32-bit column, each
+    // inside the columns its own warpgroup reads: P^T over S^T columns cb + 32 wg ..
+    // + 31 (0-31 and 96-127), dS^T likewise over the dP^T columns.  So neither warpgroup
+    // overwrites a column the other has yet to read.
+    const int wg = warp >> 2;
+    const int qw = warp & 3;
+    const int cb = wg * 64;
     const int r = qw * 32 + lane;      // key row in the tile
     const int kpos = n * 128 + r;
     const bool key_ok = p.causal || kpos < len;
     const float c = p.scale_log2;
-    const uint32_t tS = tmem_addr(tmem, qw * 32, C::COL_S);
-    const uint32_t tP = tmem_addr(tmem, qw * 32, C::COL_DP);
-    uint8_t* ds_row = smem + C::OFF_DS + (r >> 3) * 1024 + (r & 7) * 128;
+    const uint32_t tS = tmem_addr(tmem, qw * 32, C::COL_S + cb);
+    const uint32_t tPst = tmem_addr(tmem, qw * 32, C::COL_S + cb + 32 * wg);
+    const uint32_t tP = tmem_addr(tmem, qw * 32, C::COL_DP + cb);
+    const uint32_t tDSst = tmem_addr(tmem, qw * 32, C::COL_DP + cb + 32 * wg);
+    uint8_t* ds_row = smem + C::OFF_DS + wg * 16384 + (r >> 3) * 1024 + (r & 7) * 128;
     bool ok = true;
     for (int it = 0; it < iters; ++it) {
       const int st = it & 1;
@@ -372,29 +388,25 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                                        mbar_wait(&q_full[st], (it >> 1) & 1, wc, kSiteQFull));
       if (!ok) break;
       tc_fence_after();
-      const float* lse_t = lse_s + st * 128;
-      const float* dlt_t = delta_s + st * 128;
-      float pr[128];
+      const float* lse_t = lse_s + st * 128 + cb;
+      const float* dlt_t = delta_s + st * 128 + cb;
+      float pr[64];
       {
-        uint32_t u0[32], u1[32], u2[32], u3[32];
+        uint32_t u0[32], u1[32];
         tmem_ld32(tS + 0, u0);
         tmem_ld32(tS + 32, u1);
-        tmem_ld32(tS + 64, u2);
-        tmem_ld32(tS + 96, u3);
         tmem_wait_ld();
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           pr[i] = __uint_as_float(u0[i]);
           pr[32 + i] = __uint_as_float(u1[i]);
-          pr[64 + i] = __uint_as_float(u2[i]);
-          pr[96 + i] = __uint_as_float(u3[i]);
         }
       }
       const bool diag = p.causal && m == n;
       const float4* lse4 = reinterpret_cast<const float4*>(lse_t);
       const uint64_t cc = f2_pack(c, c);
 #pragma unroll
-      for (int i4 = 0; i4 < 32; ++i4) {
+      for (int i4 = 0; i4 < 16; ++i4) {
         const float4 l4 = lse4[i4];
         float x0, x1, x2, x3;
         f2_unpack(f2_fma(f2_pack(pr[4 * i4], pr[4 * i4 + 1]), cc, f2_pack(-l4.x, -l4.y)), x0, x1);
@@ -404,15 +416,15 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         for (int u = 0; u < 4; ++u) {
           const int i = 4 * i4 + u;
           const float e = ex2_approx(xv[u]);
-          pr[i] = (key_ok && !(diag && i < r)) ? e : 0.f;
+          pr[i] = (key_ok && !(diag && cb + i < r)) ? e : 0.f;
         }
       }
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
+      for (int ch = 0; ch < 2; ++ch) {
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(pr[ch * 32 + 2 * i], pr[ch * 32 + 2 * i + 1]);
-        tmem_st16(tS + ch * 16, pk);
+        tmem_st16(tPst + ch * 16, pk);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -426,11 +438,15 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                                        (it == 0 || mbar_wait(dq_full, (it - 1) & 1, wc, kSiteDqFull)));
       if (!ok) break;
       tc_fence_after();
-#pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        uint32_t u[32];
-        tmem_ld32(tP + ch * 32, u);
+      uint32_t u[64];
+      {
+        uint32_t* u0 = u;
+        tmem_ld32(tP + 0, *reinterpret_cast<uint32_t(*)[32]>(u0));
+        tmem_ld32(tP + 32, *reinterpret_cast<uint32_t(*)[32]>(u0 + 32));
         tmem_wait_ld();
+      }
+#pragma unroll
+      for (int ch = 0; ch < 2; ++ch) {
         uint32_t pk[16];
         const float4* dl4 = reinterpret_cast<const float4*>(dlt_t + ch * 32);
 #pragma unroll
@@ -439,21 +455,21 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           const int c0 = ch * 32 + 4 * i4;
           float a0, a1, a2, a3;
           f2_unpack(f2_mul(f2_pack(pr[c0], pr[c0 + 1]),
-                           f2_add(f2_pack(__uint_as_float(u[4 * i4]), __uint_as_float(u[4 * i4 + 1])),
+                           f2_add(f2_pack(__uint_as_float(u[c0]), __uint_as_float(u[c0 + 1])),
                                   f2_pack(-d4.x, -d4.y))), a0, a1);
           f2_unpack(f2_mul(f2_pack(pr[c0 + 2], pr[c0 + 3]),
-                           f2_add(f2_pack(__uint_as_float(u[4 * i4 + 2]), __uint_as_float(u[4 * i4 + 3])),
+                           f2_add(f2_pack(__uint_as_float(u[c0 + 2]), __uint_as_float(u[c0 + 3])),
                                   f2_pack(-d4.z, -d4.w))), a2, a3);
           pk[2 * i4] = pack_bf16x2(a0, a1);
           pk[2 * i4 + 1] = pack_bf16x2(a2, a3);
         }
-        tmem_st16(tP + ch * 16, pk);
-        // shared memory: query rows ch*32 .. ch*32+31 -> 64-row block ch/2, 16-byte chunks
-        uint8_t* blk = ds_row + (ch >> 1) * 16384;
+        tmem_st16(tDSst + ch * 16, pk);
+        // shared memory: this warpgroup's 64 query rows are 64-row block wg; local rows
+        // ch*32 .. ch*32+31 are 16-byte chunks ch*4 .. ch*4+3 of the key row's line
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
-          const int chunk = (ch & 1) * 4 + q4;
-          *reinterpret_cast<uint4*>(blk + ((chunk ^ (r & 7)) << 4)) =
+          const int chunk = ch * 4 + q4;
+          *reinterpret_cast<uint4*>(ds_row + ((chunk ^ (r & 7)) << 4)) =
               make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
         }
       }
@@ -463,22 +479,23 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       __syncwarp();
       if (lane == 0) mbar_arrive(ds_full);
     }
-    // epilogue: dV rows
+    // epilogue: dV rows (warps 0-3), dK rows scaled (warps 4-7)
     if (ok) {
       ok = __all_sync(0xffffffffu, mbar_wait(dkv_final, 0, wc, kSiteFinal));
       if (ok) {
         tc_fence_after();
-        const uint32_t tV = tmem_addr(tmem, qw * 32, C::COL_DV);
-        __nv_bfloat16* dst = p.dv + (size_t(start + kpos) * p.Hkv + g) * D;
+        const uint32_t tO = tmem_addr(tmem, qw * 32, wg == 0 ? C::COL_DV : C::COL_DK);
+        const float mul = wg == 0 ? 1.f : p.scale;
+        __nv_bfloat16* dst = (wg == 0 ? p.dv : p.dk) + (size_t(start + kpos) * p.Hkv + g) * D;
 #pragma unroll 1
         for (int ch = 0; ch < D / 32; ++ch) {
-          uint32_t u[32];
-          tmem_ld32(tV + ch * 32, u);
+          uint32_t v32[32];
+          tmem_ld32(tO + ch * 32, v32);
           tmem_wait_ld();
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i)
-            pk[i] = pack_bf16x2(__uint_as_float(u[2 * i]), __uint_as_float(u[2 * i + 1]));
+            pk[i] = pack_bf16x2(__uint_as_float(v32[2 * i]) * mul, __uint_as_float(v32[2 * i + 1]) * mul);
           if (kpos < len) {
             uint4* d4 = reinterpret_cast<uint4*>(dst + ch * 32);
 #pragma unroll
@@ -490,15 +507,18 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
   } else {
     reg_alloc<kRegsCompute>();
-    // ------------------------------------------------------------ dQ drain (warps 4-7)
+    // ------------------------------------------------------------ dQ drain (warps 8-11)
     // Per query tile: read dQ_tile from TMEM (thread = row), free those columns, and
     // add the rows into the fp32 workspace tile with vector reductions.  In the tile
     // layout [D/4][128][4] the 32 rows of a warp are 32 consecutive 16-byte chunks, so
     // each warp-wide reduction covers 512 contiguous bytes (four full lines), and the
-    // reductions are fire-and-forget: nothing else waits for them.
+    // reductions are fire-and-forget: nothing else waits for them.  The tile is read in
+    // two halves (register budget): the first half's reductions are issued before the
+    // second half is read and the columns are freed.
     const int qw = warp & 3;
-    const int r = qw * 32 + lane;      // query row of the tile (dQ) / key row (dK epilogue)
+    const int r = qw * 32 + lane;      // query row of the tile
     const uint32_t tQ = tmem_addr(tmem, qw * 32, C::COL_DQ);
+    constexpr int HALF = D / 2;
     bool ok = true;
     for (int it = 0; it < iters; ++it) {
       const int hq = g * p.G + it % p.G;
@@ -506,50 +526,24 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       ok = __all_sync(0xffffffffu, mbar_wait(dq_full, it & 1, wc, kSiteDqFull));
       if (!ok) break;
       tc_fence_after();
-      uint32_t acc[D];
-#pragma unroll
-      for (int ch = 0; ch < D / 32; ++ch) {
-        uint32_t u[32];
-        tmem_ld32(tQ + ch * 32, u);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) acc[ch * 32 + i] = u[i];
-      }
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(dq_free);
       float4* gdst = reinterpret_cast<float4*>(p.dq_acc + (size_t(hq) * p.ntile + tile_base + m) * 128 * D);
 #pragma unroll
-      for (int c4 = 0; c4 < D / 4; ++c4)
-        atomicAdd(gdst + c4 * 128 + r,
-                  make_float4(__uint_as_float(acc[4 * c4]), __uint_as_float(acc[4 * c4 + 1]),
-                              __uint_as_float(acc[4 * c4 + 2]), __uint_as_float(acc[4 * c4 + 3])));
-    }
-    // epilogue: dK rows (scaled)
-    if (ok) {
-      ok = __all_sync(0xffffffffu, mbar_wait(dkv_final, 0, wc, kSiteFinal));
-      if (ok) {
-        tc_fence_after();
-        const int kpos = n * 128 + r;
-        const uint32_t tK = tmem_addr(tmem, qw * 32, C::COL_DK);
-        __nv_bfloat16* dst = p.dk + (size_t(start + kpos) * p.Hkv + g) * D;
-#pragma unroll 1
-        for (int ch = 0; ch < D / 32; ++ch) {
-          uint32_t u[32];
-          tmem_ld32(tK + ch * 32, u);
-          tmem_wait_ld();
-          uint32_t pk[16];
+      for (int hf = 0; hf < 2; ++hf) {
+        uint32_t acc[HALF];
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            pk[i] = pack_bf16x2(__uint_as_float(u[2 * i]) * p.scale,
-                                __uint_as_float(u[2 * i + 1]) * p.scale);
-          if (kpos < len) {
-            uint4* d4 = reinterpret_cast<uint4*>(dst + ch * 32);
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-              d4[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
-          }
+        for (int ch = 0; ch < HALF / 32; ++ch)
+          tmem_ld32(tQ + hf * HALF + ch * 32, *reinterpret_cast<uint32_t(*)[32]>(acc + ch * 32));
+        tmem_wait_ld();
+        if (hf == 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(dq_free);
         }
+#pragma unroll
+        for (int c4 = 0; c4 < HALF / 4; ++c4)
+          atomicAdd(gdst + (hf * HALF / 4 + c4) * 128 + r,
+                    make_float4(__uint_as_float(acc[4 * c4]), __uint_as_float(acc[4 * c4 + 1]),
+                                __uint_as_float(acc[4 * c4 + 2]), __uint_as_float(acc[4 * c4 + 3])));
       }
     }
   }
