@@ -212,18 +212,30 @@ WsLayout ws_layout(int B, int Hq, long long T, int D) {
 }
 
 // Split plan of decode: tiles per split and splits per (sequence, kv head), a function
-// of the shapes only (so the workspace size needs no device query).  Aims at about two
-// CTAs per SM of a 148-SM B200 in total, at least four 128-key tiles per split, and at
-// most decode_max_parts() partial results.
+// of the shapes only (so the workspace size needs no device query).  Aims at about four
+// CTAs per SM of a 148-SM B200 in total (one CTA is resident per SM, so later CTAs fill
+// the gaps that uneven sequence lengths leave), with at least four 128-key tiles per
+// split.  When that gives less than two waves, one exact wave is better: every CTA then
+// starts at once and no SM waits on a second round.  At most decode_max_parts()
+// partial results.  (Measured on 16 x 16K-32K keys: 140 us with this plan, 161 us with
+// two CTAs per SM; on one 32K sequence: 34 us in one wave, 38 us in 1.7 waves.)
 constexpr int kPlanSMs = 148;
 int decode_max_parts() { return merge::kMaxStridedParts; }
 void decode_plan(int B, int Hkv, int Lmax, int* nsplit, int* tps) {
   const long long ntile = (Lmax + 127) / 128;
   const long long units = (long long)B * Hkv;
-  long long t = (units * ntile + 2 * kPlanSMs - 1) / (2 * kPlanSMs);
+  long long t = (units * ntile + 4 * kPlanSMs - 1) / (4 * kPlanSMs);
   if (t < 4) t = 4;
   if (t > ntile) t = ntile;
   long long ns = (ntile + t - 1) / t;
+  if (units * ns < 2 * kPlanSMs) {
+    long long ns1 = kPlanSMs / units;
+    if (ns1 < 1) ns1 = 1;
+    t = (ntile + ns1 - 1) / ns1;
+    if (t < 4) t = 4;
+    if (t > ntile) t = ntile;
+    ns = (ntile + t - 1) / t;
+  }
   if (2 * ns > decode_max_parts()) {
     ns = decode_max_parts() / 2;
     t = (ntile + ns - 1) / ns;
@@ -521,20 +533,12 @@ attn_status attn_decode(const void* q, const void* k_cache, const void* v_cache,
   mp.H = 1;
   mp.S = rows;
   mp.rows = rows;
-  const int var = merge::variant_for(w.nparts);
-  const unsigned rows_per_block =
-      unsigned(merge::kThreads / (D / 8)) * unsigned(merge::kVariantRows[var]);
-  const unsigned need = (rows + rows_per_block - 1) / rows_per_block;
-  const unsigned wave = dev->merge_grid[D == 64 ? 0 : 1][var];
-  const dim3 grid(need < wave ? need : wave);
-  const unsigned thr = merge::kThreads;
-  if (D == 64) {
-    if (var == 1) merge::attn_merge_kernel<64, 2, 2><<<grid, thr, 0, s>>>(mp);
-    else merge::attn_merge_kernel<64, 4, 1><<<grid, thr, 0, s>>>(mp);
-  } else {
-    if (var == 1) merge::attn_merge_kernel<128, 2, 2><<<grid, thr, 0, s>>>(mp);
-    else merge::attn_merge_kernel<128, 4, 1><<<grid, thr, 0, s>>>(mp);
-  }
+  // One block per (sequence, head) row: the partials of a row are spread over the
+  // block's threads, so many splits do not serialise on one thread's loads.
+  if (D == 64)
+    merge::attn_merge_rows_kernel<64><<<rows, merge::kWideThreads, 0, s>>>(mp);
+  else
+    merge::attn_merge_rows_kernel<128><<<rows, merge::kWideThreads, 0, s>>>(mp);
   return check_launch("attn_merge_kernel launch (decode)");
 }
 
