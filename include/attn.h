@@ -178,6 +178,13 @@ attn_status attn_merge(const void* const* o_parts, const float* const* lse_parts
 attn_status attn_transpose_blocks(const void* in, void* out, long long n_outer, long long n_inner,
                                   long long block_bytes, void* stream);
 
+/* Self-test of the e4m3 (fp8) tensor-core operand layouts (no page counterpart), D = 128,
+ * one 128 x 128 tile; a, b are DEVICE e4m3 bytes [128][128], pin/pq/c DEVICE fp32:
+ *   mode 3: c = a . b^T                          (both K-major)
+ *   mode 4: c = e4m3(256 pin) . b, pq = e4m3(256 pin) read back as fp32 (b MN-major) */
+attn_status attn_selftest_umma_fp8(int mode, const void* a, const void* b, const float* pin,
+                                   float* pq, float* c, void* stream);
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char* attn_strerror(attn_status status);
 

@@ -54,6 +54,7 @@ _SIGNATURES = {
     "attn_check_cu_seqlens": (_i, [ctypes.POINTER(ctypes.c_int32), _i, _i]),
     "attn_selftest_wait_timeout": (_i, [ctypes.c_ulonglong, _vp]),
     "attn_selftest_umma": (_i, [_i, _i, _vp, _vp, _fp, _vp, _fp, _vp]),
+    "attn_selftest_umma_fp8": (_i, [_i, _vp, _vp, _fp, _fp, _fp, _vp]),
     "attn_version": (_i, []),
     "attn_last_error": (ctypes.c_char_p, []),
     "attn_decode_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
@@ -180,6 +181,10 @@ def attn_selftest_wait_timeout(ns: int, stream=None) -> int:
 
 def attn_selftest_umma(mode, D, a, b, p, at, c, stream=None) -> int:
     return lib().attn_selftest_umma(mode, D, a, b, p, at, c, stream)
+
+
+def attn_selftest_umma_fp8(mode, a, b, pin, pq, c, stream=None) -> int:
+    return lib().attn_selftest_umma_fp8(mode, a, b, pin, pq, c, stream)
 
 
 def attn_version() -> int:

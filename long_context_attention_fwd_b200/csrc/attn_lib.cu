@@ -179,6 +179,19 @@ attn_status make_map(CUtensorMap* m, const void* base, int D, int H, long long T
   return r == CUDA_SUCCESS ? ATTN_OK : fail_cu("cuTensorMapEncodeTiled", r);
 }
 
+// 3-D view (D, H, T) of a [T][H][D] 1-byte (e4m3) tensor; box 128 x 1 x 128, 128-byte swizzle.
+attn_status make_map_u8(CUtensorMap* m, const void* base, int D, int H, long long T) {
+  const cuuint64_t dims[3] = {cuuint64_t(D), cuuint64_t(H), cuuint64_t(T)};
+  const cuuint64_t strides[2] = {cuuint64_t(D), cuuint64_t(H) * D};
+  const cuuint32_t box[3] = {128, 1, 128};
+  const cuuint32_t es[3] = {1, 1, 1};
+  const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims,
+                              strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ATTN_OK : fail_cu("cuTensorMapEncodeTiled (u8)", r);
+}
+
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 attn_status check_sizes(int B, int Hq, int Hkv, int S, int D, float scale, bool varlen,
@@ -640,6 +653,24 @@ extern "C" attn_status attn_selftest_umma(int mode, int D, const void* a, const 
     selftest::umma_selftest_kernel<128><<<1, 128, 32768 + 128 * 128 * 2 + 2048, s>>>(
         ma, mb, mode, pin, static_cast<const __nv_bfloat16*>(at), c, dev->status, to);
   return check_launch("umma_selftest_kernel launch");
+}
+
+extern "C" attn_status attn_selftest_umma_fp8(int mode, const void* a, const void* b,
+                                              const float* pin, float* pq, float* c, void* stream) {
+  if (mode != 3 && mode != 4) return ATTN_ERR_INVALID_ARG;
+  if (!b || !c || (mode == 3 && !a) || (mode == 4 && (!pin || !pq))) return ATTN_ERR_INVALID_ARG;
+  if (!aligned(b, 16) || (a && !aligned(a, 16)) || (pin && !aligned(pin, 16)) ||
+      (pq && !aligned(pq, 16)) || !aligned(c, 16))
+    return ATTN_ERR_MISALIGNED;
+  DeviceState* dev = nullptr;
+  attn_status st = device_setup(&dev, b);
+  if (st != ATTN_OK) return st;
+  CUtensorMap ma, mb;
+  if (make_map_u8(&ma, a ? a : b, 128, 1, 128) || make_map_u8(&mb, b, 128, 1, 128))
+    return ATTN_ERR_CUDA;
+  selftest::umma_selftest_fp8_kernel<<<1, 128, 2 * 128 * 128 + 2048, static_cast<cudaStream_t>(stream)>>>(
+      ma, mb, mode, pin, pq, c, dev->status, g_timeout_ns.load());
+  return check_launch("umma_selftest_fp8_kernel launch");
 }
 
 // ------------------------------------------------------------------ backward without allocation

@@ -123,5 +123,105 @@ umma_selftest_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_cons
   }
 }
 
+// e4m3 (kind::f8f6f4) layouts at D = 128, one 128 x 128 tile:
+//   mode 3  C = A8 B8^T                A, B e4m3 [128 rows][128], K-major via TMA: four
+//                                      MMAs of K = 32 (the S = Q K^T MMA of the fp8 forward)
+//   mode 4  C = e4m3(256 P) V8          P fp32 [128][128] quantised and packed four per TMEM
+//                                      column by the threads, V e4m3 [128 keys][128] MN-major
+//                                      via TMA (the O += P V MMA); pq receives the e4m3 values
+//                                      of 256 P as the threads read them back.
+__global__ void __launch_bounds__(128, 1)
+umma_selftest_fp8_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                         int mode, const float* __restrict__ pin, float* __restrict__ pq,
+                         float* __restrict__ cout, unsigned* status, unsigned long long timeout_ns) {
+  constexpr int TILE = 128 * 128;  // bytes of one e4m3 tile
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* sa = smem;
+  uint8_t* sb = smem + TILE;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 2 * TILE);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 3);
+  const int warp = threadIdx.x >> 5, r = threadIdx.x;
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    mbar_init(&bars[0], 1);
+    mbar_init(&bars[1], 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const WaitCtl wc{status, abort_flag, timeout_ns};
+
+  if (threadIdx.x == 0) {
+    mbar_arrive_expect_tx(&bars[0], (mode == 3 ? TILE : 0) + TILE);
+    if (mode == 3) tma_load_3d(&tm_a, &bars[0], sa, 0, 0, 0);
+    tma_load_3d(&tm_b, &bars[0], sb, 0, 0, 0);
+  }
+  if (mode == 4) {
+    // P row r -> TMEM lane r, columns 128..159: four e4m3 keys per 32-bit column
+    const uint32_t tp = tmem_addr(tmem, warp * 32, 128);
+    for (int ch = 0; ch < 2; ++ch) {
+      uint32_t pk[16];
+      for (int i = 0; i < 16; ++i) {
+        const float* x = pin + r * 128 + ch * 64 + 4 * i;
+        pk[i] = pack_e4m3x2(256.f * x[0], 256.f * x[1]) | (pack_e4m3x2(256.f * x[2], 256.f * x[3]) << 16);
+        float a0, a1, a2, a3;
+        unpack_e4m3x2(pk[i], a0, a1);
+        unpack_e4m3x2(pk[i] >> 16, a2, a3);
+        float* q = pq + r * 128 + ch * 64 + 4 * i;
+        q[0] = a0; q[1] = a1; q[2] = a2; q[3] = a3;
+      }
+      tmem_st16(tp + ch * 16, pk);
+    }
+    tmem_wait_st();
+  }
+  tc_fence_before();
+  __syncthreads();
+  bool ok = true;
+  if (threadIdx.x == 0) {
+    ok = mbar_wait(&bars[0], 0, wc, 0x310);
+    if (ok) {
+      tc_fence_after();
+      const uint32_t ab = smem_u32(sa), bb = smem_u32(sb);
+      if (mode == 3) {
+        constexpr uint32_t id = idesc_e4m3_f32(128, 128, 0, 0);
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ss_f8(tmem, sdesc_sw128(ab + kk * 32, 16, 1024), sdesc_sw128(bb + kk * 32, 16, 1024), id, kk > 0);
+      } else {
+        constexpr uint32_t id = idesc_e4m3_f32(128, 128, 0, 1);
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ts_f8(tmem, tmem + 128 + kk * 8, sdesc_sw128(bb + kk * 4096, 16384, 1024), id, kk > 0);
+      }
+    }
+    mma_commit(&bars[1]);
+  }
+  ok = __all_sync(0xffffffffu, mbar_wait(&bars[1], 0, wc, 0x311));
+  if (ok) {
+    tc_fence_after();
+    const uint32_t tc = tmem_addr(tmem, warp * 32, 0);
+    for (int ch = 0; ch < 4; ++ch) {
+      uint32_t u[32];
+      tmem_ld32(tc + ch * 32, u);
+      tmem_wait_ld();
+      for (int i = 0; i < 32; ++i) cout[r * 128 + ch * 32 + i] = __uint_as_float(u[i]);
+    }
+  }
+  if (threadIdx.x == 0) mbar_drain(&bars[0], 0, timeout_ns);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
 }  // namespace selftest
 }  // namespace attn_sm100

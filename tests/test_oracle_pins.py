@@ -410,3 +410,21 @@ def test_decode_gqa_and_ignores_entries_past_the_length():
     k2[0, 7:], v2[0, 7:] = 1e30, np.nan
     o3, l3 = oracle.decode(q, k2, v2, lens, 0.5)
     assert np.array_equal(o1, o3) and np.array_equal(l1, l3)
+
+
+# ---------------------------------------------------------------- e4m3 helper used by the fp8 tests
+def test_e4m3_helper_against_the_format():
+    import e4m3
+    # every finite code decodes to a value that quantises back to itself
+    codes = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], dtype=np.uint8)
+    vals = e4m3.decode(codes)
+    np.testing.assert_array_equal(e4m3.quantize(vals), vals)
+    assert e4m3.decode(np.array([0x7E], np.uint8))[0] == 448.0          # largest finite
+    assert e4m3.decode(np.array([0x01], np.uint8))[0] == 2.0 ** -9      # smallest subnormal
+    assert e4m3.decode(np.array([0x08], np.uint8))[0] == 2.0 ** -6      # smallest normal
+    assert np.isnan(e4m3.decode(np.array([0x7F], np.uint8))[0])
+    # ties go to the even mantissa; saturation at 448
+    assert e4m3.quantize(1.0 + 1.0 / 16) == 1.0           # halfway 1.0 / 1.125 -> even (1.0)
+    assert e4m3.quantize(1.0 + 3.0 / 16) == 1.25          # halfway 1.125 / 1.25 -> even (1.25)
+    assert e4m3.quantize(1000.0) == 448.0 and e4m3.quantize(-1000.0) == -448.0
+    assert e4m3.quantize(2.0 ** -10) == 0.0               # halfway 0 / 2^-9 -> even (0)
