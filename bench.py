@@ -16,7 +16,8 @@ On one GPU the line also carries "ring": the exact merge kernel of Ring attentio
 4-rank ring run rank after rank on this GPU; and "ulysses": the relayout kernel around
 the Ulysses all-to-alls (HBM-bound) and forward + backward of a 4-rank Ulysses group run
 rank after rank on this GPU; and "decode": attention of one new token per sequence over
-a 32K-token KV cache (HBM-bound).  All are measured after the timed steps.
+a 32K-token KV cache (HBM-bound); and "fp8_fwd": the e4m3 forward on the bench workload.
+All are measured after the timed steps.
 
 --impl reference times the fp64 CPU oracle (the reference arm of this build) on a
 bounded sample of the same workload: the first tokens of the causal sequence form
@@ -347,6 +348,45 @@ def ulysses_measurements(wr: I.Workload, q, k, v, do, stream, peaks, world=4, re
     }
 
 
+def fp8_measurements(wr: I.Workload, q, k, v, stream, peaks, reps=10):
+    """Measures the e4m3 forward (attn_fwd_fp8) on the bench workload, outside the timed
+    step: the bf16 inputs quantised per tensor (descale = max|x| / 448) on the GPU, then
+    forward TFLOP/s (same FLOP convention) against the fp8 peak, taken as the measured bf16
+    peak times the nominal fp8 : bf16 ratio of 2 (4.5 vs 2.25 PFLOP/s dense)."""
+    import torch
+    from long_context_attention_fwd_b200 import ops
+
+    def q8(t):
+        d = float(t.abs().max().float()) / 448.0
+        return (t.float() / d).clamp_(-448.0, 448.0).to(torch.float8_e4m3fn), d
+
+    (q8_, qd), (k8_, kd), (v8_, vd) = q8(q), q8(k), q8(v)
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(reps)]
+        torch.cuda.synchronize()
+        for e0, e1 in evs:
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        return statistics.median(e0.elapsed_time(e1) for e0, e1 in evs)
+
+    fp8_ms = timed(lambda: ops.attn_fwd_fp8(q8_, k8_, v8_, qd, kd, vd, causal=wr.causal,
+                                            scale=wr.softmax_scale))
+    bf16_ms = timed(lambda: ops.attn_fwd(q, k, v, causal=wr.causal, scale=wr.softmax_scale))
+    tf = I.flop_fwd(wr) / (fp8_ms * 1e-3) / 1e12
+    peak = 2.0 * float(peaks.get("bf16_tflops"))
+    return {"kernel": "attn_fwd_kernel<128, e4m3>", "bound": "tensor", "ms": fp8_ms,
+            "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
+            "peak_source": "MEASURED_PEAKS.json bf16_tflops (burst) x 2, the nominal fp8:bf16 ratio",
+            "bf16_fwd_ms_same_run": bf16_ms, "speedup_vs_bf16": bf16_ms / fp8_ms,
+            "inputs": "the bench workload's q, k, v quantised per tensor to e4m3 on the GPU"}
+
+
 def decode_measurements(dev, stream, peaks, reps=20):
     """Measures decode attention over a KV cache (attn_decode: split-KV kernel + merge) on
     the two decode workloads, outside the timed step.  HBM-bound: achieved = the cached
@@ -520,6 +560,9 @@ def run_gpu(args, w: I.Workload):
     if (ws == 1 and dense and wr.S % 4 == 0 and wr.Hq % 4 == 0 and wr.Hkv % 4 == 0
             and not args.no_ulysses):
         uly_rows = ulysses_measurements(wr, q, k, v, do, stream, peaks)
+    fp8_row = None
+    if ws == 1 and dense and wr.D == 128 and not args.no_fp8:
+        fp8_row = fp8_measurements(wr, q, k, v, stream, peaks)
     dec_rows = None
     if ws == 1 and not args.no_decode:
         dec_rows = decode_measurements(dev, stream, peaks)
@@ -559,6 +602,8 @@ def run_gpu(args, w: I.Workload):
             line["ulysses"] = uly_rows
         if dec_rows is not None:
             line["decode"] = dec_rows
+        if fp8_row is not None:
+            line["fp8_fwd"] = fp8_row
         if ws == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(wr)
         print(json.dumps(line), flush=True)
@@ -577,6 +622,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-fp8", action="store_true",
+                    help="skip the e4m3 forward measurement")
     ap.add_argument("--no-decode", action="store_true",
                     help="skip the decode-attention measurements")
     ap.add_argument("--no-ulysses", action="store_true",

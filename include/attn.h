@@ -63,6 +63,23 @@ attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float
                      int Hq, int Hkv, int S, int D, int causal, float scale,
                      const int32_t* cu_seqlens, void* stream);
 
+/* FP8 forward (page "ms-swift集成FlashAttention 2/3，长文本训练更高效", section
+ * "FlashAttention 如何破局": FlashAttention-3 adds FP8 computation on Hopper; this is the
+ * same idea on B200's fifth-generation tensor cores).  q, k, v hold e4m3 values (1 byte,
+ * same [T][H][D] layouts as attn_fwd) with per-tensor descale factors: the attention of
+ * (q_descale * q, k_descale * k, v_descale * v) is computed, i.e.
+ *     s_ij = scale * q_descale * k_descale * (q8_i . k8_j),   o_i = v_descale * sum_j P_ij v8_j.
+ * The probabilities are quantised for the P V product as e4m3(256 p) (the factor keeps
+ * probabilities down to 2^-14 in e4m3's normal range and cancels in the normalisation,
+ * which divides by the sum of exactly the quantised weights).  o is bf16, lse fp32 as in
+ * attn_fwd (computed from the unquantised probabilities).  D must be 128
+ * (ATTN_ERR_UNSUPPORTED otherwise); descale factors and their product with scale must be
+ * finite.  Everything else (masks, GQA, packed batches, errors) as attn_fwd. */
+attn_status attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                         int Hq, int Hkv, int S, int D, int causal, float scale, float q_descale,
+                         float k_descale, float v_descale, const int32_t* cu_seqlens,
+                         void* stream);
+
 /* Bytes of device workspace attn_bwd needs for these arguments (same meaning as in
  * attn_bwd; only whether cu_seqlens is NULL matters).  Holds, per query head and
  * 128-row query tile, the fp32 dQ accumulator tile, Delta = rowsum(dO * O) and

@@ -45,6 +45,8 @@ _sz = ctypes.c_size_t
 
 _SIGNATURES = {
     "attn_fwd": (_i, [_vp, _vp, _vp, _vp, _fp, _i, _i, _i, _i, _i, _i, ctypes.c_float, _vp, _vp]),
+    "attn_fwd_fp8": (_i, [_vp, _vp, _vp, _vp, _fp, _i, _i, _i, _i, _i, _i, ctypes.c_float,
+                          ctypes.c_float, ctypes.c_float, ctypes.c_float, _vp, _vp]),
     "attn_bwd_workspace_size": (_sz, [_i, _i, _i, _i, _vp]),
     "attn_bwd": (_i, [_vp, _vp, _vp, _vp, _fp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
                       ctypes.c_float, _vp, _vp, _sz, _vp]),
@@ -113,6 +115,13 @@ def check(status: int, where: str) -> None:
 def attn_fwd(q, k, v, o, lse, B, Hq, Hkv, S, D, causal, scale, cu_seqlens, stream) -> int:
     return lib().attn_fwd(q, k, v, o, lse, B, Hq, Hkv, S, D, int(causal), float(scale),
                           cu_seqlens, stream)
+
+
+def attn_fwd_fp8(q, k, v, o, lse, B, Hq, Hkv, S, D, causal, scale, q_descale, k_descale,
+                 v_descale, cu_seqlens, stream) -> int:
+    return lib().attn_fwd_fp8(q, k, v, o, lse, B, Hq, Hkv, S, D, int(causal), float(scale),
+                              float(q_descale), float(k_descale), float(v_descale), cu_seqlens,
+                              stream)
 
 
 def attn_bwd_workspace_size(B, Hq, S, D, cu_seqlens) -> int:

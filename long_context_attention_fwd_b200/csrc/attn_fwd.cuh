@@ -19,6 +19,12 @@
 //               more than 2^8, and finally normalises O and stores O and LSE.
 // The two tiles ping-pong: while softmax works on one tile the tensor core runs the
 // other tile's PV and the next S, so MMA and exponentials overlap.
+//
+// FP8 = true is the e4m3 variant (D = 128): Q, K, V are e4m3 with per-tensor descale
+// factors folded into the softmax scale (q, k) and the epilogue (v); the MMAs are
+// kind::f8f6f4 (K = 32 per instruction, twice the bf16 rate); P is quantised as
+// e4m3(256 p) -- the factor 256 keeps probabilities down to 2^-14 in e4m3's normal range
+// -- and O is divided by the sum of exactly those quantised weights, so the factor cancels.
 #pragma once
 #include <cuda_bf16.h>
 #include "attn_common.cuh"
@@ -47,17 +53,27 @@ struct Params {
   float* lse;
   int Hq, G, T;                        // query heads, query heads per kv head, total tokens
   int causal;
-  float scale_log2;                    // softmax scale * log2(e)
+  float scale_log2;                    // softmax scale * log2(e) (* q, k descale for e4m3)
+  float o_scale;                       // 1, or the v descale for e4m3
   int nblk;                            // (T >> 8) + nseq: upper bound of 256-row blocks
   unsigned* status;
   unsigned long long timeout_ns;
 };
 
-template <int D>
+constexpr float kP8Scale = 256.0f;      // e4m3 P = e4m3(256 p)
+// e4m3 saturates at 448, so 256 p must stay below it: p is relative to the running maximum,
+// which the lazy rescale lets lag the true one by up to the threshold.  2^0.5 * 256 = 362.
+constexpr float kRescaleThresholdFp8 = 0.5f;
+
+template <int D, bool FP8 = false>
 struct Cfg {
-  static constexpr int NS = (D == 128) ? 2 : 4;
-  static constexpr int QT_BYTES = BM * D * 2;
-  static constexpr int KV_BYTES = BN * D * 2;
+  static constexpr int ES = FP8 ? 1 : 2;                 // bytes per element
+  static constexpr int NS = FP8 ? 4 : ((D == 128) ? 2 : 4);
+  static constexpr int SLABS = D * ES / 128;             // 128-byte swizzle rows per tile row
+  static constexpr int KSTEPS = D * ES / 32;             // MMAs over D (32 bytes of K each)
+  static constexpr int PSTEPS = BN * ES / 32;            // MMAs over the keys of a tile
+  static constexpr int QT_BYTES = BM * D * ES;
+  static constexpr int KV_BYTES = BN * D * ES;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + 2 * QT_BYTES;
   static constexpr int OFF_V = OFF_K + NS * KV_BYTES;
@@ -77,11 +93,12 @@ enum : unsigned {
   kSiteOFinal
 };
 
-template <int D>
+template <int D, bool FP8 = false>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const Params p) {
-  using C = Cfg<D>;
+  static_assert(!FP8 || D == 128, "the e4m3 variant is built for D = 128");
+  using C = Cfg<D, FP8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
 
@@ -160,24 +177,24 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       mbar_arrive_expect_tx(q_full, qbytes);
       for (int t = 0; t < 2; ++t) {
         if (n_t[t] == 0) continue;
-        for (int hf = 0; hf < D / 64; ++hf)
-          tma_load_3d(&tm_q, q_full, smem + C::OFF_Q + t * C::QT_BYTES + hf * kSlab, hf * 64, h,
-                      start + q_row0 + BM * t);
+        for (int hf = 0; hf < C::SLABS; ++hf)
+          tma_load_3d(&tm_q, q_full, smem + C::OFF_Q + t * C::QT_BYTES + hf * kSlab,
+                      hf * (128 / C::ES), h, start + q_row0 + BM * t);
       }
       for (int j = 0; j < jmax; ++j) {
         const int st = j % C::NS;
         const uint32_t ph = (j / C::NS) & 1;
         if (!mbar_wait(&k_empty[st], ph ^ 1, wc, kSiteKEmpty)) break;
         mbar_arrive_expect_tx(&k_full[st], C::KV_BYTES);
-        for (int hf = 0; hf < D / 64; ++hf)
+        for (int hf = 0; hf < C::SLABS; ++hf)
           tma_load_3d(&tm_k, &k_full[st], smem + C::OFF_K + st * C::KV_BYTES + hf * kSlab,
-                      hf * 64, g, start + BN * j);
+                      hf * (128 / C::ES), g, start + BN * j);
         ++nk;
         if (!mbar_wait(&v_empty[st], ph ^ 1, wc, kSiteVEmpty)) break;
         mbar_arrive_expect_tx(&v_full[st], C::KV_BYTES);
-        for (int hf = 0; hf < D / 64; ++hf)
+        for (int hf = 0; hf < C::SLABS; ++hf)
           tma_load_3d(&tm_v, &v_full[st], smem + C::OFF_V + st * C::KV_BYTES + hf * kSlab,
-                      hf * 64, g, start + BN * j);
+                      hf * (128 / C::ES), g, start + BN * j);
         ++nv;
       }
       // Drain: every issued copy must land before shared memory is released.
@@ -192,26 +209,35 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
    } else if (warp == kWarpMMA) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idS = idesc_bf16_f32(128, 128, 0, 0);
-      constexpr uint32_t idPV = idesc_bf16_f32(128, D, 0, 1);
+      constexpr uint32_t idS = FP8 ? idesc_e4m3_f32(128, 128, 0, 0) : idesc_bf16_f32(128, 128, 0, 0);
+      constexpr uint32_t idPV = FP8 ? idesc_e4m3_f32(128, D, 0, 1) : idesc_bf16_f32(128, D, 0, 1);
       const uint32_t qb[2] = {smem_u32(smem + C::OFF_Q), smem_u32(smem + C::OFF_Q + C::QT_BYTES)};
       const uint32_t colS[2] = {C::COL_S0, C::COL_S1};
       const uint32_t colO[2] = {C::COL_O0, C::COL_O1};
       auto issue_S = [&](int t, int st) {
         const uint32_t kb = smem_u32(smem + C::OFF_K + st * C::KV_BYTES);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
+        for (int kk = 0; kk < C::KSTEPS; ++kk) {
           const uint32_t off = (kk >> 2) * kSlab + (kk & 3) * 32;
-          mma_ss(tmem + colS[t], sdesc_sw128(qb[t] + off, 16, 1024),
-                 sdesc_sw128(kb + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
+          if constexpr (FP8)
+            mma_ss_f8(tmem + colS[t], sdesc_sw128(qb[t] + off, 16, 1024),
+                      sdesc_sw128(kb + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
+          else
+            mma_ss(tmem + colS[t], sdesc_sw128(qb[t] + off, 16, 1024),
+                   sdesc_sw128(kb + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
         }
       };
       auto issue_PV = [&](int t, int st, bool acc) {
         const uint32_t vb = smem_u32(smem + C::OFF_V + st * C::KV_BYTES);
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk)
-          mma_ts(tmem + colO[t], tmem + colS[t] + kk * 8, sdesc_sw128(vb + kk * 2048, kSlab, 1024),
-                 idPV, (acc || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < C::PSTEPS; ++kk) {
+          // K step: 32 bytes of keys = 32 / ES key rows of 128 bytes in the MN-major V tile
+          const uint64_t bdesc = sdesc_sw128(vb + kk * (4096 / C::ES), kSlab, 1024);
+          if constexpr (FP8)
+            mma_ts_f8(tmem + colO[t], tmem + colS[t] + kk * 8, bdesc, idPV, (acc || kk > 0) ? 1u : 0u);
+          else
+            mma_ts(tmem + colO[t], tmem + colS[t] + kk * 8, bdesc, idPV, (acc || kk > 0) ? 1u : 0u);
+        }
       };
       bool ok = mbar_wait(q_full, 0, wc, kSiteQFull) && mbar_wait(&k_full[0], 0, wc, kSiteKFull);
       if (ok) {
@@ -323,7 +349,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         mx = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]);
       }
       const float mx2 = mx * c;
-      const bool need = mx2 > m_run + kRescaleThreshold;
+      const bool need = mx2 > m_run + (FP8 ? kRescaleThresholdFp8 : kRescaleThreshold);
       const float m_new = need ? mx2 : m_run;
       const float alpha = need ? ex2_approx(m_run - m_new) : 1.f;
       if (j > 0 && __any_sync(0xffffffffu, need)) {
@@ -346,6 +372,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       // their bf16 roundings (the values the PV MMA consumes), so that O is
       // normalised by exactly the weights it was accumulated with.
       uint64_t sf[4] = {0, 0, 0, 0}, sb[4] = {0, 0, 0, 0};
+      if constexpr (!FP8) {
 #pragma unroll
       for (int ch = 0; ch < 4; ++ch) {
         uint32_t pk[16];
@@ -360,6 +387,31 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           sb[i & 3] = f2_add(sb[i & 3], f2_pack(__uint_as_float(b << 16), __uint_as_float(b & 0xFFFF0000u)));
         }
         tmem_st16(tS + ch * 16, pk);
+      }
+      } else {
+        // e4m3: four keys per 32-bit column, 256 p quantised; sb sums the quantised values
+#pragma unroll
+        for (int ch = 0; ch < 2; ++ch) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int k0 = ch * 64 + 4 * i;
+            float x0, x1, x2, x3;
+            f2_unpack(f2_fma(f2_pack(s[k0], s[k0 + 1]), cc, mm), x0, x1);
+            f2_unpack(f2_fma(f2_pack(s[k0 + 2], s[k0 + 3]), cc, mm), x2, x3);
+            const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+            const float p2 = ex2_approx(x2), p3 = ex2_approx(x3);
+            const uint32_t lo = pack_e4m3x2(kP8Scale * p0, kP8Scale * p1);
+            const uint32_t hi = pack_e4m3x2(kP8Scale * p2, kP8Scale * p3);
+            pk[i] = lo | (hi << 16);
+            float q0, q1, q2, q3;
+            unpack_e4m3x2(lo, q0, q1);
+            unpack_e4m3x2(hi, q2, q3);
+            sf[i & 3] = f2_add(sf[i & 3], f2_add(f2_pack(p0, p1), f2_pack(p2, p3)));
+            sb[i & 3] = f2_add(sb[i & 3], f2_add(f2_pack(q0, q1), f2_pack(q2, q3)));
+          }
+          tmem_st16(tS + ch * 16, pk);
+        }
       }
       {
         float a0, a1, b0, b1;
@@ -377,7 +429,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       ok = __all_sync(0xffffffffu, mbar_wait(&o_final[t], 0, wc, kSiteOFinal));
       if (ok) {
         tc_fence_after();
-        const float inv = 1.f / lb_run;
+        // lb_run sums the weights the PV MMA used (for e4m3 in units of 1/256, which the
+        // division cancels); o_scale is 1, or the v descale.
+        const float inv = p.o_scale / lb_run;
         const bool valid = rpos < len;
         __nv_bfloat16* orow = p.o + (size_t(start + rpos) * p.Hq + h) * D;
 #pragma unroll 1

@@ -106,6 +106,7 @@ attn_status device_setup(DeviceState** out, const void* ptr = nullptr) {
       cudaError_t e = cudaSuccess;
       e = e ? e : cudaFuncSetAttribute(fwd::attn_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, fwd::Cfg<64>::SMEM_ALLOC);
       e = e ? e : cudaFuncSetAttribute(fwd::attn_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, fwd::Cfg<128>::SMEM_ALLOC);
+      e = e ? e : cudaFuncSetAttribute(fwd::attn_fwd_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, fwd::Cfg<128, true>::SMEM_ALLOC);
       e = e ? e : cudaFuncSetAttribute(bwd::attn_bwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, bwd::Cfg<64>::SMEM_ALLOC);
       e = e ? e : cudaFuncSetAttribute(bwd::attn_bwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, bwd::Cfg<128>::SMEM_ALLOC);
       e = e ? e : cudaFuncSetAttribute(decode::attn_decode_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, decode::Cfg<64>::SMEM_ALLOC);
@@ -115,16 +116,18 @@ attn_status device_setup(DeviceState** out, const void* ptr = nullptr) {
       if (e != cudaSuccess) return fail_cuda("cudaFuncSetAttribute", e);
       // The kernels re-split registers between warpgroups with setmaxnreg; that is only
       // safe when each thread starts with exactly the budget the split was sized for.
-      const void* split_kernels[6] = {
+      const void* split_kernels[7] = {
           reinterpret_cast<const void*>(fwd::attn_fwd_kernel<64>),
           reinterpret_cast<const void*>(fwd::attn_fwd_kernel<128>),
+          reinterpret_cast<const void*>(fwd::attn_fwd_kernel<128, true>),
           reinterpret_cast<const void*>(bwd::attn_bwd_kernel<64>),
           reinterpret_cast<const void*>(bwd::attn_bwd_kernel<128>),
           reinterpret_cast<const void*>(decode::attn_decode_kernel<64>),
           reinterpret_cast<const void*>(decode::attn_decode_kernel<128>)};
-      const int split_regs[6] = {fwd::kRegsLaunch, fwd::kRegsLaunch, bwd::kRegsLaunch,
-                                 bwd::kRegsLaunch, decode::kRegsLaunch, decode::kRegsLaunch};
-      for (int i = 0; i < 6; ++i) {
+      const int split_regs[7] = {fwd::kRegsLaunch, fwd::kRegsLaunch, fwd::kRegsLaunch,
+                                 bwd::kRegsLaunch, bwd::kRegsLaunch, decode::kRegsLaunch,
+                                 decode::kRegsLaunch};
+      for (int i = 0; i < 7; ++i) {
         cudaFuncAttributes fa;
         if ((e = cudaFuncGetAttributes(&fa, split_kernels[i])) != cudaSuccess)
           return fail_cuda("cudaFuncGetAttributes", e);
@@ -336,6 +339,7 @@ attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float
   p.T = int(T);
   p.causal = causal ? 1 : 0;
   p.scale_log2 = scale * 1.4426950408889634f;
+  p.o_scale = 1.f;
   p.nblk = int((T >> 8) + B);
   p.status = dev->status;
   p.timeout_ns = g_timeout_ns.load();
@@ -346,6 +350,45 @@ attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float
   else
     fwd::attn_fwd_kernel<128><<<grid, fwd::kThreads, fwd::Cfg<128>::SMEM_ALLOC, s>>>(mq, mk, mv, p);
   return check_launch("attn_fwd_kernel launch");
+}
+
+attn_status attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                         int Hq, int Hkv, int S, int D, int causal, float scale, float q_descale,
+                         float k_descale, float v_descale, const int32_t* cu_seqlens,
+                         void* stream) {
+  long long T = 0;
+  attn_status st = check_sizes(B, Hq, Hkv, S, D, scale, cu_seqlens != nullptr, &T);
+  if (st != ATTN_OK) return st;
+  if (D != 128) return ATTN_ERR_UNSUPPORTED;
+  if (!std::isfinite(q_descale) || !std::isfinite(k_descale) || !std::isfinite(v_descale) ||
+      !std::isfinite(scale * q_descale * k_descale))
+    return ATTN_ERR_INVALID_ARG;
+  if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+      !aligned(lse, 4) || (cu_seqlens && !aligned(cu_seqlens, 4)))
+    return ATTN_ERR_MISALIGNED;
+  DeviceState* dev = nullptr;
+  if ((st = device_setup(&dev, q)) != ATTN_OK) return st;
+  CUtensorMap mq, mk, mv;
+  if (make_map_u8(&mq, q, D, Hq, T) || make_map_u8(&mk, k, D, Hkv, T) || make_map_u8(&mv, v, D, Hkv, T))
+    return ATTN_ERR_CUDA;
+  fwd::Params p;
+  p.sv = SeqView{cu_seqlens, B, cu_seqlens ? int(T) : S, int(T)};
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.Hq = Hq;
+  p.G = Hq / Hkv;
+  p.T = int(T);
+  p.causal = causal ? 1 : 0;
+  p.scale_log2 = scale * q_descale * k_descale * 1.4426950408889634f;
+  p.o_scale = v_descale;
+  p.nblk = int((T >> 8) + B);
+  p.status = dev->status;
+  p.timeout_ns = g_timeout_ns.load();
+  const dim3 grid(unsigned(p.nblk) * unsigned(Hq));
+  fwd::attn_fwd_kernel<128, true><<<grid, fwd::kThreads, fwd::Cfg<128, true>::SMEM_ALLOC,
+                                    static_cast<cudaStream_t>(stream)>>>(mq, mk, mv, p);
+  return check_launch("attn_fwd_kernel<fp8> launch");
 }
 
 size_t attn_bwd_workspace_size(int B, int Hq, int S, int D, const int32_t* cu_seqlens) {

@@ -6,6 +6,7 @@
     o = attention(q, k, v, causal=True)                        # autograd-aware
     o, lse = attn_merge([o1, o2], [lse1, lse2])                # exact merge of key-chunk partials
     o, lse = attn_decode(q, k_cache, v_cache, cache_len)       # one new token per sequence
+    o, lse = attn_fwd_fp8(q8, k8, v8, qd, kd, vd)              # e4m3 inputs + descale factors
 
 All arithmetic runs in libattn.so; these functions only check shapes, allocate
 outputs with torch and pass raw pointers and the current CUDA stream.
@@ -226,4 +227,38 @@ def attn_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
                           cache_len.data_ptr(), out.data_ptr(), lse.data_ptr(), B, Hq, Hkv, Lmax,
                           D, scale, workspace.data_ptr(), workspace.numel(), _stream(q.device))
     capi.check(st, "attn_decode")
+    return out, lse
+
+
+def _check_e4m3(*ts: torch.Tensor) -> None:
+    for t in ts:
+        if not t.is_cuda:
+            raise ValueError("libattn needs CUDA tensors (there is no CPU path)")
+        if t.dtype not in (torch.float8_e4m3fn, torch.uint8):
+            raise ValueError("fp8 tensors must be float8_e4m3fn (or their bytes as uint8)")
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+
+
+def attn_fwd_fp8(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, q_descale: float,
+                 k_descale: float, v_descale: float, causal: bool = True,
+                 scale: Optional[float] = None, cu_seqlens: Optional[torch.Tensor] = None,
+                 out: Optional[torch.Tensor] = None,
+                 lse: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """e4m3 forward: attention of (q_descale q, k_descale k, v_descale v), D = 128.
+    Returns (o bf16, lse fp32) in attn_fwd's layouts."""
+    _check_e4m3(q, k, v)
+    B, S, Hq, Hkv, D = _dims(q, k, cu_seqlens)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        shape = (Hq, S) if cu_seqlens is not None else (B, Hq, S)
+        lse = torch.empty(shape, dtype=torch.float32, device=q.device)
+    st = capi.attn_fwd_fp8(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                           B, Hq, Hkv, S, D, causal, scale, q_descale, k_descale, v_descale,
+                           cu_seqlens.data_ptr() if cu_seqlens is not None else None,
+                           _stream(q.device))
+    capi.check(st, "attn_fwd_fp8")
     return out, lse

@@ -33,3 +33,22 @@ def random_bytes(rng, shape, max_exp: int = 9) -> np.ndarray:
     e = rng.integers(1, max_exp + 1, size=shape) << 3
     m = rng.integers(0, 8, size=shape)
     return (s | e | m).astype(np.uint8)
+
+
+def encode(q: np.ndarray) -> np.ndarray:
+    """Bytes of values that are already e4m3 numbers (e.g. quantize's output)."""
+    q = np.asarray(q, dtype=np.float64)
+    s = (q < 0).astype(np.int64) << 7
+    a = np.abs(q)
+    sub = a < 2.0 ** -6
+    e = np.where(sub, 0, np.floor(np.log2(np.where(sub, 1.0, a))) + 7).astype(np.int64)
+    m = np.where(sub, np.rint(a / 2.0 ** -9), np.rint((a / np.exp2(e - 7.0) - 1.0) * 8.0)).astype(np.int64)
+    return (s | (e << 3) | m).astype(np.uint8)
+
+
+def quantize_tensor(x: np.ndarray):
+    """Per-tensor scaling as FP8 attention uses it: descale = max|x| / 448, bytes of
+    e4m3(x / descale).  Returns (bytes, descale)."""
+    amax = float(np.abs(x).max())
+    descale = amax / E4M3_MAX if amax > 0 else 1.0
+    return encode(quantize(x / descale)), descale

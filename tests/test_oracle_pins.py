@@ -428,3 +428,6 @@ def test_e4m3_helper_against_the_format():
     assert e4m3.quantize(1.0 + 3.0 / 16) == 1.25          # halfway 1.125 / 1.25 -> even (1.25)
     assert e4m3.quantize(1000.0) == 448.0 and e4m3.quantize(-1000.0) == -448.0
     assert e4m3.quantize(2.0 ** -10) == 0.0               # halfway 0 / 2^-9 -> even (0)
+    # encoding is the inverse of decoding on every finite code (except -0 -> +0)
+    enc = e4m3.encode(vals)
+    assert all(a == b or (a == 0x80 and b == 0) for a, b in zip(codes, enc))
