@@ -14,6 +14,8 @@ Parity status per function (pins live in tests/test_oracle_pins.py):
   invariants, finite differences and hand-derived golden values;
   merge_partials -- pinned by "merging chunk partials equals attention over all keys"
   and its special cases;
+  bwd_given -- pinned by summing its block-pair gradients over a ring split and comparing
+  with PyTorch's fp64 autograd of the whole attention;
   decode -- pinned by PyTorch's fp64 attention routine, closed forms (V = ones, identical
   keys, one cached key, an empty cache) and grouped-query = repeated multi-head.
 """
@@ -77,6 +79,9 @@ def _load():
             lib.oracle_attn_bwd_dkdv_range.argtypes = [_D] * 4 + common + [
                 ctypes.c_int] * 4 + [_D, _D]
             lib.oracle_num_threads.restype = ctypes.c_int
+            lib.oracle_attn_bwd_given.argtypes = [_D, _D, _D, _D, _D, _D, _D, _D, _D, ctypes.c_int,
+                                                  ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                  ctypes.c_int, ctypes.c_int, ctypes.c_double]
             lib.oracle_attn_decode.argtypes = [_D, _D, _D, _I32, _D, _D, ctypes.c_int,
                                                ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                                ctypes.c_int, ctypes.c_double]
@@ -252,3 +257,20 @@ def decode(q, k_cache, v_cache, cache_len, scale: float):
     if rc:
         raise ValueError(f"oracle_attn_decode failed ({rc})")
     return o, lse
+
+
+def bwd_given(q, k, v, o, lse, do, causal: bool, scale: float, B: int, S: int):
+    """Block-pair backward with the whole problem's O [B*S,Hq,D] and LSE [B,Hq,S] given
+    -> (dq, dk, dv); dense layouts as in bwd."""
+    q, k, v, o, lse, do = (_f64(x) for x in (q, k, v, o, lse, do))
+    T, Hq, D = q.shape
+    Hkv = k.shape[1]
+    if T != B * S or lse.shape != (B, Hq, S) or o.shape != q.shape or do.shape != q.shape:
+        raise ValueError("shapes do not match")
+    dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    rc = _load().oracle_attn_bwd_given(_dp(q), _dp(k), _dp(v), _dp(o), _dp(lse), _dp(do), _dp(dq),
+                                       _dp(dk), _dp(dv), B, Hq, Hkv, S, D, int(causal),
+                                       float(scale))
+    if rc:
+        raise ValueError(f"oracle_attn_bwd_given failed ({rc})")
+    return dq, dk, dv

@@ -538,3 +538,77 @@ int oracle_attn_decode(const double *q, const double *k_cache, const double *v_c
     }
     return err;
 }
+
+/*
+ * Backward of one query/key block pair of a larger attention, given the FULL problem's row
+ * statistics (page "ms-swift集成FlashAttention 2/3，长文本训练更高效", section "单靠
+ * FlashAttention 不够？那就加上序列并行", subsection "Ring-Attention": with the sequence
+ * split across devices, each device computes the part of the result its own queries and the
+ * passing key/value block contribute).  With O and LSE of the whole row, the block's share
+ * of the gradient is exactly:
+ *     P_ij = exp(scale q_i . k_j - LSE_i),  Delta_i = dO_i . O_i,
+ *     dS_ij = P_ij (dO_i . v_j - Delta_i),
+ *     dQ_i += scale sum_j dS_ij k_j,  dK_j += scale sum_i dS_ij q_i,  dV_j += sum_i P_ij dO_i,
+ * summed over the query heads of each kv head; summing the blocks gives the full gradient.
+ * Dense batches: q, o, dout, dq [B*S][Hq][D]; k, v, dk, dv [B*S][Hkv][D]; lse [B][Hq][S].
+ * causal masks key j for query i when j > i (positions within the block pair: the diagonal
+ * block of a causal split).  Outputs are overwritten.
+ */
+int oracle_attn_bwd_given(const double *q, const double *k, const double *v, const double *o,
+                          const double *lse, const double *dout, double *dq, double *dk, double *dv,
+                          int B, int Hq, int Hkv, int S, int D, int causal, double scale) {
+    if (B < 1 || Hq < 1 || Hkv < 1 || S < 1 || D < 1 || Hq % Hkv) return 1;
+    const int G = Hq / Hkv;
+    memset(dq, 0, sizeof(double) * (size_t)B * S * Hq * D);
+    memset(dk, 0, sizeof(double) * (size_t)B * S * Hkv * D);
+    memset(dv, 0, sizeof(double) * (size_t)B * S * Hkv * D);
+    /* dQ: parallel over query rows */
+#pragma omp parallel for schedule(dynamic, 4)
+    for (int64_t r = 0; r < (int64_t)B * S * Hq; ++r) {
+        const int64_t t = r / Hq;
+        const int h = (int)(r % Hq), b = (int)(t / S), i = (int)(t % S), g = h / G;
+        const double *qi = q + r * D, *oi = o + r * D, *doi = dout + r * D;
+        double delta = 0.0;
+        for (int d = 0; d < D; ++d) delta += doi[d] * oi[d];
+        const double L = lse[((int64_t)b * Hq + h) * S + i];
+        double *dqi = dq + r * D;
+        const int n = causal ? i + 1 : S;
+        for (int j = 0; j < n; ++j) {
+            const double *kj = k + (((int64_t)b * S + j) * Hkv + g) * D;
+            const double *vj = v + (((int64_t)b * S + j) * Hkv + g) * D;
+            double s = 0.0, dp = 0.0;
+            for (int d = 0; d < D; ++d) { s += qi[d] * kj[d]; dp += doi[d] * vj[d]; }
+            const double p = exp(scale * s - L);
+            const double ds = p * (dp - delta);
+            for (int d = 0; d < D; ++d) dqi[d] += scale * ds * kj[d];
+        }
+    }
+    /* dK, dV: parallel over key rows */
+#pragma omp parallel for schedule(dynamic, 4)
+    for (int64_t c = 0; c < (int64_t)B * S * Hkv; ++c) {
+        const int64_t t = c / Hkv;
+        const int g = (int)(c % Hkv), b = (int)(t / S), j = (int)(t % S);
+        const double *kj = k + c * D, *vj = v + c * D;
+        double *dkj = dk + c * D, *dvj = dv + c * D;
+        for (int hh = 0; hh < G; ++hh) {
+            const int h = g * G + hh;
+            for (int i = causal ? j : 0; i < S; ++i) {
+                const int64_t r = ((int64_t)b * S + i) * Hq + h;
+                const double *qi = q + r * D, *oi = o + r * D, *doi = dout + r * D;
+                double delta = 0.0, s = 0.0, dp = 0.0;
+                for (int d = 0; d < D; ++d) {
+                    delta += doi[d] * oi[d];
+                    s += qi[d] * kj[d];
+                    dp += doi[d] * vj[d];
+                }
+                const double p = exp(scale * s - lse[((int64_t)b * Hq + h) * S + i]);
+                const double ds = p * (dp - delta);
+                for (int d = 0; d < D; ++d) {
+                    dkj[d] += scale * ds * qi[d];
+                    dvj[d] += p * doi[d];
+                }
+            }
+        }
+    }
+    return 0;
+}

@@ -125,3 +125,23 @@ def test_decode_validation_and_workspace():
     assert d(A, A, A, A + 2, A, A, 2, 8, 2, 512, 64, 0.125, A, need, None) == capi.ATTN_ERR_MISALIGNED
     assert d(A, A, A, A, A, A, 2, 8, 2, 512, 96, 0.125, A, need, None) == capi.ATTN_ERR_UNSUPPORTED
     assert d(A, A, A, A, A, A, 2, 8, 2, 512, 64, float("nan"), A, need, None) == capi.ATTN_ERR_INVALID_ARG
+
+
+def test_fwd_fp8_validation():
+    f = capi.attn_fwd_fp8
+    ok = (A, A, A, A, A, 1, 8, 2, 256, 128, 1, 0.125, 0.01, 0.02, 0.03, None, None)
+    assert f(*ok[:9], 64, *ok[10:]) == capi.ATTN_ERR_UNSUPPORTED               # D must be 128
+    assert f(*ok[:12], float("nan"), *ok[13:]) == capi.ATTN_ERR_INVALID_ARG      # q descale
+    assert f(*ok[:14], float("inf"), *ok[15:]) == capi.ATTN_ERR_INVALID_ARG      # v descale
+    assert f(*ok[:12], 1e30, 1e30, *ok[14:]) == capi.ATTN_ERR_INVALID_ARG        # scale product
+    assert f(None, *ok[1:]) == capi.ATTN_ERR_INVALID_ARG
+    assert f(A + 8, *ok[1:]) == capi.ATTN_ERR_MISALIGNED
+    assert f(*ok[:5], 1, 6, 4, 256, 128, *ok[10:]) == capi.ATTN_ERR_INVALID_ARG  # Hq % Hkv
+
+
+def test_selftest_fp8_validation():
+    t = capi.attn_selftest_umma_fp8
+    assert t(2, A, A, A, A, A, None) == capi.ATTN_ERR_INVALID_ARG
+    assert t(3, None, A, None, None, A, None) == capi.ATTN_ERR_INVALID_ARG       # mode 3 needs a
+    assert t(4, None, A, None, A, A, None) == capi.ATTN_ERR_INVALID_ARG          # mode 4 needs pin
+    assert t(3, A, A + 8, None, None, A, None) == capi.ATTN_ERR_MISALIGNED

@@ -32,6 +32,7 @@ MUTANTS = {
                                   "const double w = exp(lse_parts[p][r] - m);"),
     "merge_lse_without_max": ("const double L = m + log(sum);", "const double L = log(sum);"),
     "decode_drops_last_key": ("const int L = cache_len[b];", "const int L = cache_len[b] > 1 ? cache_len[b] - 1 : cache_len[b];"),
+    "bwd_given_ignores_lse": ("const double p = exp(scale * s - L);", "const double p = exp(scale * s);"),
     "decode_gqa_map_modulo": ("const int b = (int)(r / Hq), h = (int)(r % Hq), g = h / G;",
                               "const int b = (int)(r / Hq), h = (int)(r % Hq), g = h % Hkv;"),
 }
@@ -109,6 +110,30 @@ def _pin_suite() -> list:
         ok &= abs(ld[0, h] - (s_.max() + np.log(e.sum()))) < 1e-12
     if not ok:
         failed.append("decode_direct")
+    # block-pair backward with the whole rows' statistics: the two-block causal split sums
+    # to PyTorch's fp64 autograd of the whole attention
+    try:
+        import torch
+        C, Hq5, Hkv5, D5, sc = 5, 2, 1, 3, 0.7
+        S5 = 2 * C
+        q5, k5, v5, do5 = _rnd((S5, Hq5, D5), 31), _rnd((S5, Hkv5, D5), 32), _rnd((S5, Hkv5, D5), 33), _rnd((S5, Hq5, D5), 34)
+        o5, l5 = oracle.fwd(q5, k5, v5, True, sc, B=1, S=S5)
+        g = [np.zeros_like(q5), np.zeros_like(k5), np.zeros_like(v5)]
+        for r in range(2):
+            qs = slice(r * C, (r + 1) * C)
+            for j in range(r + 1):
+                ks = slice(j * C, (j + 1) * C)
+                a, b_, c_ = oracle.bwd_given(q5[qs], k5[ks], v5[ks], o5[qs], l5[:, :, qs], do5[qs], j == r, sc, B=1, S=C)
+                g[0][qs] += a; g[1][ks] += b_; g[2][ks] += c_
+        tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q5, k5, v5))
+        out = torch.nn.functional.scaled_dot_product_attention(
+            tq.permute(1, 0, 2)[None], tk.repeat_interleave(2, 1).permute(1, 0, 2)[None],
+            tv.repeat_interleave(2, 1).permute(1, 0, 2)[None], is_causal=True, scale=sc)[0].permute(1, 0, 2)
+        out.backward(torch.tensor(do5))
+        if not all(np.allclose(a, b_.grad.numpy(), atol=1e-10) for a, b_ in zip(g, (tq, tk, tv))):
+            failed.append("bwd_given_sum")
+    except ValueError:
+        failed.append("bwd_given_sum")
     # finite differences of L = sum(dO * O)
     S2 = 5
     q, k, v, do = _rnd((S2, 2, 3), 6), _rnd((S2, 1, 3), 7), _rnd((S2, 1, 3), 8), _rnd((S2, 2, 3), 9)

@@ -431,3 +431,30 @@ def test_e4m3_helper_against_the_format():
     # encoding is the inverse of decoding on every finite code (except -0 -> +0)
     enc = e4m3.encode(vals)
     assert all(a == b or (a == 0x80 and b == 0) for a, b in zip(codes, enc))
+
+
+# ---------------------------------------------------------------- block-pair backward (Ring)
+def test_bwd_given_block_pairs_sum_to_torch_autograd():
+    torch = pytest.importorskip("torch")
+    C, Hq, Hkv, D, scale = 9, 4, 2, 4, 0.6
+    S = 2 * C
+    q, k, v, do = rnd((S, Hq, D), 101), rnd((S, Hkv, D), 102), rnd((S, Hkv, D), 103), rnd((S, Hq, D), 104)
+    o, lse = oracle.fwd(q, k, v, True, scale, B=1, S=S)          # statistics of the whole rows
+    dq = np.zeros_like(q); dk = np.zeros_like(k); dv = np.zeros_like(v)
+    for r in range(2):                                           # query block r
+        qs = slice(r * C, (r + 1) * C)
+        for j in range(r + 1):                                   # key blocks it sees
+            ks = slice(j * C, (j + 1) * C)
+            gq, gk, gv = oracle.bwd_given(q[qs], k[ks], v[ks], o[qs], lse[:, :, qs], do[qs],
+                                          j == r, scale, B=1, S=C)
+            dq[qs] += gq; dk[ks] += gk; dv[ks] += gv
+    G = Hq // Hkv
+    tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+    kk = tk.repeat_interleave(G, dim=1); vv = tv.repeat_interleave(G, dim=1)
+    out = torch.nn.functional.scaled_dot_product_attention(
+        tq.permute(1, 0, 2)[None], kk.permute(1, 0, 2)[None], vv.permute(1, 0, 2)[None],
+        is_causal=True, scale=scale)[0].permute(1, 0, 2)
+    out.backward(torch.tensor(do))
+    np.testing.assert_allclose(dq, tq.grad.numpy(), atol=1e-11)
+    np.testing.assert_allclose(dk, tk.grad.numpy(), atol=1e-11)
+    np.testing.assert_allclose(dv, tv.grad.numpy(), atol=1e-11)
