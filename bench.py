@@ -273,6 +273,12 @@ def ring_measurements(wr: I.Workload, q, k, v, o, lse, stream, peaks, world=4, r
                                                              wr.softmax_scale))
     fwd_ms = timed(lambda: ops.attn_fwd(q, k, v, causal=wr.causal, scale=wr.softmax_scale))
     del o_parts, lse_parts, out, lse_out
+    do = torch.randn(q.shape, device=q.device, dtype=torch.float32).to(q.dtype)
+    ring_bwd_ms = timed(lambda: ring.ring_attn_bwd_single_device(q, k, v, o, lse, do, world,
+                                                                 wr.causal, wr.softmax_scale))
+    bwd_ms = timed(lambda: ops.attn_bwd(q, k, v, o, lse, do, causal=wr.causal,
+                                        scale=wr.softmax_scale))
+    del do
     n_fwd = sum(len(ring.ring_schedule(r, world, wr.causal)) for r in range(world))
     n_merge = sum(len(ring.ring_schedule(r, world, wr.causal)) > 1 for r in range(world))
     return {
@@ -290,6 +296,12 @@ def ring_measurements(wr: I.Workload, q, k, v, o, lse, stream, peaks, world=4, r
                              "attn_merge_launches": n_merge,
                              "note": "every rank's partials and merge run one after another on "
                                      "this GPU; the K/V transfers of a real ring are not timed"},
+        "ring_bwd_one_gpu": {"world": world, "ms": ring_bwd_ms,
+                             "tflops": I.flop_bwd(wr) / (ring_bwd_ms * 1e-3) / 1e12,
+                             "single_kernel_bwd_ms": bwd_ms,
+                             "note": "block-pair attn_bwd with the merged O/LSE per scheduled pair, "
+                                     "shares summed in fp32 (attn_accumulate_bf16), rounded once; "
+                                     "every rank on this GPU, transfers not timed"},
     }
 
 

@@ -177,6 +177,19 @@ attn_status attn_decode(const void* q, const void* k_cache, const void* v_cache,
 attn_status attn_merge(const void* const* o_parts, const float* const* lse_parts, int nparts,
                        void* o, float* lse, int B, int H, int S, int D, void* stream);
 
+/* Accumulation of block gradients for the Ring-Attention backward (page
+ * "ms-swift集成FlashAttention 2/3，长文本训练更高效", section "单靠 FlashAttention 不够？
+ * 那就加上序列并行", subsection "Ring-Attention": each device computes the share of the
+ * result its queries and the passing key/value block contribute; in the backward, the
+ * shares -- bf16 outputs of attn_bwd on each block pair -- are summed in fp32):
+ *     acc[i] = (init ? 0 : acc[i]) + x[i]        acc fp32, x bf16, i < n
+ * DEVICE pointers, 16-byte aligned; n >= 1 and a multiple of 8. */
+attn_status attn_accumulate_bf16(float* acc, const void* x, long long n, int init, void* stream);
+
+/* out[i] = bf16(in[i]) (round to nearest even): the final rounding of an fp32 accumulator
+ * (same pointer and size rules as attn_accumulate_bf16). */
+attn_status attn_convert_f32_bf16(void* out, const float* in, long long n, void* stream);
+
 /* Block transpose for the layout changes around the all-to-alls of Ulysses sequence
  * parallelism (page "ms-swift集成FlashAttention 2/3，长文本训练更高效", section "单靠
  * FlashAttention 不够？那就加上序列并行", Ulysses subsection: split the sequence across

@@ -13,7 +13,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libattn.so")
 SOURCES = ["attn_lib.cu"]
-HEADERS = ["sm100_ptx.cuh", "attn_common.cuh", "attn_fwd.cuh", "attn_bwd.cuh", "attn_decode.cuh", "attn_merge.cuh",
+HEADERS = ["sm100_ptx.cuh", "attn_accum.cuh", "attn_common.cuh", "attn_fwd.cuh", "attn_bwd.cuh", "attn_decode.cuh", "attn_merge.cuh",
            "attn_relayout.cuh",
            "umma_selftest.cuh"]
 NVCC_FLAGS = [

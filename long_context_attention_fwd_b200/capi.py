@@ -62,6 +62,8 @@ _SIGNATURES = {
     "attn_decode_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
     "attn_decode": (_i, [_vp, _vp, _vp, _vp, _vp, _fp, _i, _i, _i, _i, _i, ctypes.c_float, _vp,
                          _sz, _vp]),
+    "attn_accumulate_bf16": (_i, [_fp, _vp, ctypes.c_longlong, _i, _vp]),
+    "attn_convert_f32_bf16": (_i, [_vp, _fp, ctypes.c_longlong, _vp]),
     "attn_transpose_blocks": (_i, [_vp, _vp, ctypes.c_longlong, ctypes.c_longlong,
                                    ctypes.c_longlong, _vp]),
     "attn_merge": (_i, [_vp, _vp, _i, _vp, _fp, _i, _i, _i, _i, _vp]),
@@ -159,6 +161,14 @@ def attn_decode(q, k_cache, v_cache, cache_len, o, lse, B, Hq, Hkv, Lmax, D, sca
                 workspace_bytes, stream) -> int:
     return lib().attn_decode(q, k_cache, v_cache, cache_len, o, lse, B, Hq, Hkv, Lmax, D,
                              float(scale), workspace, workspace_bytes, stream)
+
+
+def attn_accumulate_bf16(acc, x, n, init, stream) -> int:
+    return lib().attn_accumulate_bf16(acc, x, int(n), int(init), stream)
+
+
+def attn_convert_f32_bf16(out, inp, n, stream) -> int:
+    return lib().attn_convert_f32_bf16(out, inp, int(n), stream)
 
 
 def attn_transpose_blocks(inp, out, n_outer, n_inner, block_bytes, stream) -> int:

@@ -12,6 +12,7 @@
 #include <mutex>
 
 #include "../../include/attn.h"
+#include "attn_accum.cuh"
 #include "attn_bwd.cuh"
 #include "attn_decode.cuh"
 #include "attn_fwd.cuh"
@@ -59,6 +60,7 @@ struct DeviceState {
   unsigned* status = nullptr;
   unsigned merge_grid[2][merge::kVariants] = {};  // resident blocks per merge kernel (D 64/128)
   unsigned relayout_grid = 0;                     // resident blocks of transpose_blocks_kernel
+  unsigned sms = 0;                               // SM count (grid size of element-wise kernels)
 };
 std::mutex g_mu;
 DeviceState g_dev[kMaxDevices];
@@ -162,6 +164,7 @@ attn_status device_setup(DeviceState** out, const void* ptr = nullptr) {
         d.relayout_grid = unsigned(prop.multiProcessorCount) * unsigned(per_sm > 0 ? per_sm : 1);
       }
     }
+    d.sms = unsigned(prop.multiProcessorCount);
     d.ready = true;
   }
   if (!d.sm100) return ATTN_ERR_UNSUPPORTED;
@@ -596,6 +599,38 @@ attn_status attn_decode(const void* q, const void* k_cache, const void* v_cache,
   else
     merge::attn_merge_rows_kernel<128><<<rows, merge::kWideThreads, 0, s>>>(mp);
   return check_launch("attn_merge_kernel launch (decode)");
+}
+
+attn_status attn_accumulate_bf16(float* acc, const void* x, long long n, int init, void* stream) {
+  if (!acc || !x || n < 1) return ATTN_ERR_INVALID_ARG;
+  if (n % 8) return ATTN_ERR_INVALID_ARG;
+  if (!aligned(acc, 16) || !aligned(x, 16)) return ATTN_ERR_MISALIGNED;
+  DeviceState* dev = nullptr;
+  attn_status st = device_setup(&dev, acc);
+  if (st != ATTN_OK) return st;
+  const long long n8 = n / 8;
+  const long long need = (n8 + accum::kThreads - 1) / accum::kThreads;
+  const long long wave = (long long)dev->sms * 8;
+  accum::add_bf16_to_f32_kernel<<<unsigned(need < wave ? need : wave), accum::kThreads, 0,
+                                  static_cast<cudaStream_t>(stream)>>>(
+      reinterpret_cast<float4*>(acc), static_cast<const uint4*>(x), n8, init ? 1 : 0);
+  return check_launch("add_bf16_to_f32_kernel launch");
+}
+
+attn_status attn_convert_f32_bf16(void* out, const float* in, long long n, void* stream) {
+  if (!out || !in || n < 1) return ATTN_ERR_INVALID_ARG;
+  if (n % 8) return ATTN_ERR_INVALID_ARG;
+  if (!aligned(out, 16) || !aligned(in, 16)) return ATTN_ERR_MISALIGNED;
+  DeviceState* dev = nullptr;
+  attn_status st = device_setup(&dev, in);
+  if (st != ATTN_OK) return st;
+  const long long n8 = n / 8;
+  const long long need = (n8 + accum::kThreads - 1) / accum::kThreads;
+  const long long wave = (long long)dev->sms * 8;
+  accum::f32_to_bf16_kernel<<<unsigned(need < wave ? need : wave), accum::kThreads, 0,
+                              static_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint4*>(out), reinterpret_cast<const float4*>(in), n8);
+  return check_launch("f32_to_bf16_kernel launch");
 }
 
 attn_status attn_transpose_blocks(const void* in, void* out, long long n_outer, long long n_inner,

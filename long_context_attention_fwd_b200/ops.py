@@ -262,3 +262,24 @@ def attn_fwd_fp8(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, q_descale: f
                            _stream(q.device))
     capi.check(st, "attn_fwd_fp8")
     return out, lse
+
+
+def accumulate_bf16(acc: torch.Tensor, x: torch.Tensor, init: bool = False) -> torch.Tensor:
+    """acc (fp32) = (0 if init else acc) + x (bf16), element-wise in libattn.so."""
+    if not (acc.is_cuda and x.is_cuda and acc.is_contiguous() and x.is_contiguous()):
+        raise ValueError("accumulate_bf16 needs contiguous CUDA tensors (there is no CPU path)")
+    if acc.dtype != torch.float32 or x.dtype != torch.bfloat16 or acc.numel() != x.numel():
+        raise ValueError("acc must be fp32 and x bf16 of the same size")
+    capi.check(capi.attn_accumulate_bf16(acc.data_ptr(), x.data_ptr(), x.numel(), init,
+                                         _stream(x.device)), "attn_accumulate_bf16")
+    return acc
+
+
+def convert_f32_bf16(x: torch.Tensor, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """bf16 copy of an fp32 tensor (round to nearest even) in libattn.so."""
+    if not (x.is_cuda and x.is_contiguous() and x.dtype == torch.float32):
+        raise ValueError("convert_f32_bf16 needs a contiguous fp32 CUDA tensor")
+    out = torch.empty(x.shape, dtype=torch.bfloat16, device=x.device) if out is None else out
+    capi.check(capi.attn_convert_f32_bf16(out.data_ptr(), x.data_ptr(), x.numel(),
+                                          _stream(x.device)), "attn_convert_f32_bf16")
+    return out

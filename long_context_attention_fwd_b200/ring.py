@@ -18,9 +18,17 @@ and chunks j > r are skipped.  The partials are combined by the exact log-sum-ex
 
 K/V chunks travel with torch.distributed point-to-point sends (NCCL on GPUs) into local
 buffers; the kernels only ever read this GPU's own memory.
+
+Backward (ring_attn_bwd, and ring_attention for autograd): each block pair's share of the
+gradient is the block-pair backward with the whole rows' O and LSE (attn_bwd given the
+merged o and lse).  K/V chunks circulate as in the forward; the fp32 dK/dV accumulators of
+the chunk a rank holds travel with it, each rank adding its share, and return to the
+chunk's owner after N hops; dQ accumulates locally.  Shares are summed in fp32 and rounded
+to bf16 once.
 """
 from __future__ import annotations
 
+from dataclasses import dataclass
 from typing import Callable, List, Optional, Tuple
 
 import torch
@@ -123,3 +131,131 @@ def ring_attn_fwd_single_device(q: torch.Tensor, k: torch.Tensor, v: torch.Tenso
         outs.append(o)
         lses.append(lse)
     return torch.cat(outs, dim=1), torch.cat(lses, dim=2)
+
+
+@dataclass
+class RingHooks:
+    """Compute steps of the Ring forward/backward; the defaults are this library's kernels.
+    The CPU tests replace them (the fp64 oracle and plain tensor arithmetic)."""
+    fwd: Callable = None       # (q, k, v, causal, scale) -> (o, lse)
+    merge: Callable = None     # (o_parts, lse_parts) -> (o, lse)
+    bwd: Callable = None       # (q, k, v, o, lse, do, causal, scale) -> (dq, dk, dv), block pair
+    acc: Callable = None       # (acc, x, init) -> acc = (0 if init else acc) + x
+    cast: Callable = None      # (acc) -> result dtype
+    acc_dtype: torch.dtype = torch.float32
+
+    def resolved(self) -> "RingHooks":
+        return RingHooks(
+            fwd=self.fwd or _default_attend,
+            merge=self.merge or ops.attn_merge,
+            bwd=self.bwd or (lambda q, k, v, o, l, do, c, s:
+                             ops.attn_bwd(q, k, v, o, l, do, causal=c, scale=s)),
+            acc=self.acc or (lambda a, x, init: ops.accumulate_bf16(a, x, init)),
+            cast=self.cast or ops.convert_f32_bf16,
+            acc_dtype=self.acc_dtype)
+
+
+def ring_attn_bwd(q, k, v, o, lse, do, causal: bool = True, scale: Optional[float] = None,
+                  group=None, hooks: Optional[RingHooks] = None):
+    """Backward of ring_attn_fwd for this rank's chunk: o, lse are the merged forward
+    results of the local queries, do the gradient of o.  Returns (dq, dk, dv) of the local
+    chunk."""
+    import torch.distributed as dist
+
+    h = (hooks or RingHooks()).resolved()
+    world = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    if world == 1:
+        return h.bwd(q, k, v, o, lse, do, causal, scale)
+    plan = {s: (j, c) for s, j, c in ring_schedule(rank, world, causal)}
+    nxt, prv = (rank + 1) % world, (rank - 1) % world
+    if group is not None:
+        nxt, prv = dist.get_global_rank(group, nxt), dist.get_global_rank(group, prv)
+    new_acc = lambda t: torch.empty(t.shape, dtype=h.acc_dtype, device=t.device)
+    kv_bufs = [(torch.empty_like(k), torch.empty_like(v)) for _ in range(2)]
+    acc_bufs = [(new_acc(k), new_acc(v)) for _ in range(2)]
+    dq_acc = new_acc(q)
+    cur_k, cur_v = k, v
+    cur_dk, cur_dv = new_acc(k), new_acc(v)   # this rank's own chunk; initialised at step 0
+    for s in range(world):
+        kv_works = []
+        if s < world - 1:
+            nk, nv = kv_bufs[s % 2]
+            kv_works = dist.batch_isend_irecv([
+                dist.P2POp(dist.isend, cur_k, nxt, group), dist.P2POp(dist.irecv, nk, prv, group),
+                dist.P2POp(dist.isend, cur_v, nxt, group), dist.P2POp(dist.irecv, nv, prv, group)])
+        if s in plan:   # step 0 is always the diagonal block: it initialises the accumulators
+            gq, gk, gv = h.bwd(q, cur_k, cur_v, o, lse, do, plan[s][1], scale)
+            h.acc(dq_acc, gq, s == 0)
+            h.acc(cur_dk, gk, s == 0)
+            h.acc(cur_dv, gv, s == 0)
+        ndk, ndv = acc_bufs[s % 2]
+        acc_works = dist.batch_isend_irecv([
+            dist.P2POp(dist.isend, cur_dk, nxt, group), dist.P2POp(dist.irecv, ndk, prv, group),
+            dist.P2POp(dist.isend, cur_dv, nxt, group), dist.P2POp(dist.irecv, ndv, prv, group)])
+        for w in kv_works + acc_works:
+            w.wait()
+        if s < world - 1:
+            cur_k, cur_v = kv_bufs[s % 2]
+        cur_dk, cur_dv = ndk, ndv
+    # After N hops every chunk's accumulators are back with its owner.
+    return h.cast(dq_acc), h.cast(cur_dk), h.cast(cur_dv)
+
+
+class _RingAttention(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, q, k, v, causal, scale, group, hooks):
+        o, lse = ring_attn_fwd(q, k, v, causal, scale, group, attend=hooks.fwd, merge=hooks.merge)
+        ctx.save_for_backward(q, k, v, o, lse)
+        ctx.causal, ctx.scale, ctx.group, ctx.hooks = causal, scale, group, hooks
+        return o
+
+    @staticmethod
+    def backward(ctx, do):
+        q, k, v, o, lse = ctx.saved_tensors
+        dq, dk, dv = ring_attn_bwd(q, k, v, o, lse, do.contiguous(), ctx.causal, ctx.scale,
+                                   ctx.group, ctx.hooks)
+        return dq, dk, dv, None, None, None, None
+
+
+def ring_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = True,
+                   scale: Optional[float] = None, group=None,
+                   hooks: Optional[RingHooks] = None) -> torch.Tensor:
+    """Autograd-aware Ring attention of this rank's chunk (layouts as ring_attn_fwd)."""
+    return _RingAttention.apply(q, k, v, causal, scale, group, (hooks or RingHooks()).resolved())
+
+
+def ring_attn_bwd_single_device(q, k, v, o, lse, do, world: int, causal: bool = True,
+                                scale: Optional[float] = None,
+                                hooks: Optional[RingHooks] = None):
+    """Every rank's share of the Ring backward, run one after another on this device from
+    the full tensors (q/o/do [B][S][Hq][D], k/v [B][S][Hkv][D], lse [B][Hq][S]): the same
+    block-pair backwards and fp32 accumulation as ring_attn_bwd, without the transfers.
+    Returns the full (dq, dk, dv)."""
+    h = (hooks or RingHooks()).resolved()
+    S = q.shape[1]
+    if S % world:
+        raise ValueError("sequence length must be divisible by the ring size")
+    C = S // world
+
+    def chunk(t, j):
+        return t[:, j * C:(j + 1) * C].contiguous()
+
+    new_acc = lambda t: torch.empty(t.shape, dtype=h.acc_dtype, device=t.device)
+    dk_acc = [new_acc(chunk(k, j)) for j in range(world)]
+    dv_acc = [new_acc(chunk(v, j)) for j in range(world)]
+    kv_started = [False] * world          # has chunk j's accumulator received a share yet
+    dq_out = []
+    for r in range(world):
+        qr, orr, dor = chunk(q, r), chunk(o, r), chunk(do, r)
+        lr = lse[:, :, r * C:(r + 1) * C].contiguous()
+        dq_acc = new_acc(qr)
+        for s, j, c in ring_schedule(r, world, causal):
+            gq, gk, gv = h.bwd(qr, chunk(k, j), chunk(v, j), orr, lr, dor, c, scale)
+            h.acc(dq_acc, gq, s == 0)          # step 0 is every rank's first share
+            h.acc(dk_acc[j], gk, not kv_started[j])
+            h.acc(dv_acc[j], gv, not kv_started[j])
+            kv_started[j] = True
+        dq_out.append(h.cast(dq_acc))
+    return (torch.cat(dq_out, dim=1), torch.cat([h.cast(a) for a in dk_acc], dim=1),
+            torch.cat([h.cast(a) for a in dv_acc], dim=1))

@@ -117,3 +117,85 @@ def test_gloo_ring_equals_full_attention(world, causal):
     for r, err_o, err_l in res:
         assert err_o < 1e-12, (r, err_o)
         assert err_l < 1e-12, (r, err_l)
+
+
+# ---------------------------------------------------------------- backward
+def oracle_bwd_pair(q, k, v, o, lse, do, causal, scale):
+    B, C = q.shape[:2]
+    g = oracle.bwd_given(q.numpy().reshape(B * C, q.shape[2], -1), k.numpy().reshape(B * C, k.shape[2], -1),
+                         v.numpy().reshape(B * C, v.shape[2], -1), o.numpy().reshape(B * C, o.shape[2], -1),
+                         lse.numpy(), do.numpy().reshape(B * C, do.shape[2], -1), causal, scale, B=B, S=C)
+    return tuple(torch.from_numpy(np.ascontiguousarray(x)).reshape(t.shape) for x, t in zip(g, (q, k, v)))
+
+
+def _acc(a, x, init):
+    if init:
+        a.copy_(x)
+    else:
+        a.add_(x)
+    return a
+
+
+RING_HOOKS = ring.RingHooks(fwd=oracle_attend, merge=oracle_merge, bwd=oracle_bwd_pair, acc=_acc,
+                            cast=lambda a: a.clone(), acc_dtype=torch.float64)
+
+
+def _full_grads(q, k, v, do, causal, scale):
+    B, S, Hq, D = q.shape
+    tok = lambda t: t.numpy().reshape(B * S, t.shape[2], D)
+    g = oracle.bwd(tok(q), tok(k), tok(v), tok(do), causal, scale, B=B, S=S)
+    return [x.reshape(t.shape) for x, t in zip(g, (q, k, v))]
+
+
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("world", [2, 3])
+def test_single_device_backward_equals_full_gradients(causal, world):
+    B, S, Hq, Hkv, D = 2, 12 * world, 4, 2, 4
+    q, k, v = full_problem(B, S, Hq, Hkv, D, 21)
+    do = torch.from_numpy(I.normal(I.stream_key(21, 9), B * S * Hq * D).reshape(B, S, Hq, D))
+    o, lse = ring.ring_attn_fwd_single_device(q, k, v, world, causal, 0.3, attend=oracle_attend,
+                                              merge=oracle_merge)
+    dq, dk, dv = ring.ring_attn_bwd_single_device(q, k, v, o, lse, do, world, causal, 0.3,
+                                                  hooks=RING_HOOKS)
+    for got, want in zip((dq, dk, dv), _full_grads(q, k, v, do, causal, 0.3)):
+        np.testing.assert_allclose(got.numpy(), want, atol=1e-11)
+
+
+def _bwd_worker(rank, world, port, causal, q_out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        B, S, Hq, Hkv, D = 1, 8 * world, 4, 2, 4
+        q, k, v = full_problem(B, S, Hq, Hkv, D, 23)
+        do = torch.from_numpy(I.normal(I.stream_key(23, 9), B * S * Hq * D).reshape(B, S, Hq, D))
+        C = S // world
+        sl = slice(rank * C, (rank + 1) * C)
+        ql, kl, vl = (t[:, sl].contiguous().requires_grad_(True) for t in (q, k, v))
+        o = ring.ring_attention(ql, kl, vl, causal, 0.35, hooks=RING_HOOKS)
+        o.backward(do[:, sl].contiguous())
+        want = _full_grads(q, k, v, do, causal, 0.35)
+        errs = [float(np.abs(g.detach().numpy() - w_[:, sl]).max())
+                for g, w_ in zip((ql.grad, kl.grad, vl.grad), want)]
+        q_out.put((rank, errs))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,causal", [(2, True), (4, True), (3, False)])
+def test_gloo_ring_backward_equals_full_gradients(world, causal):
+    ctx = mp.get_context("spawn")
+    q_out = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_bwd_worker, args=(r, world, port, causal, q_out))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted(q_out.get(timeout=180) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for r, errs in res:
+        assert max(errs) < 1e-11, (r, errs)
