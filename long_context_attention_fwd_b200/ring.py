@@ -51,6 +51,13 @@ def ring_schedule(rank: int, world: int, causal: bool) -> List[Tuple[int, int, b
     return out
 
 
+def _check_dense(*ts) -> None:
+    for t in ts:
+        if t.dim() != 4:
+            raise ValueError("the Ring wrappers take dense [B][C][H][D] chunks (packed batches "
+                             "are not supported)")
+
+
 def _default_attend(q, k, v, causal, scale) -> Partial:
     return ops.attn_fwd(q, k, v, causal=causal, scale=scale)
 
@@ -68,6 +75,7 @@ def ring_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: boo
     """
     import torch.distributed as dist
 
+    _check_dense(q, k, v)
     attend = attend or _default_attend
     merge = merge or ops.attn_merge
     world = dist.get_world_size(group)
@@ -111,6 +119,7 @@ def ring_attn_fwd_single_device(q: torch.Tensor, k: torch.Tensor, v: torch.Tenso
     """Every rank's share of a `world`-rank ring, run one after another on this device from
     the full tensors (q [B][S][Hq][D], k/v [B][S][Hkv][D], S divisible by `world`): the same
     partials and merges as ring_attn_fwd, without the transfers.  Returns the full (o, lse)."""
+    _check_dense(q, k, v)
     attend = attend or _default_attend
     merge = merge or ops.attn_merge
     B, S = q.shape[0], q.shape[1]
@@ -162,6 +171,7 @@ def ring_attn_bwd(q, k, v, o, lse, do, causal: bool = True, scale: Optional[floa
     chunk."""
     import torch.distributed as dist
 
+    _check_dense(q, k, v, o, do)
     h = (hooks or RingHooks()).resolved()
     world = dist.get_world_size(group)
     rank = dist.get_rank(group)
@@ -232,6 +242,7 @@ def ring_attn_bwd_single_device(q, k, v, o, lse, do, world: int, causal: bool = 
     the full tensors (q/o/do [B][S][Hq][D], k/v [B][S][Hkv][D], lse [B][Hq][S]): the same
     block-pair backwards and fp32 accumulation as ring_attn_bwd, without the transfers.
     Returns the full (dq, dk, dv)."""
+    _check_dense(q, k, v, o, do)
     h = (hooks or RingHooks()).resolved()
     S = q.shape[1]
     if S % world:

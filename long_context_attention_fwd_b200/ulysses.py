@@ -47,6 +47,13 @@ class Hooks:
             transpose=self.transpose or ops.transpose_blocks)
 
 
+def check_dense(*ts) -> None:
+    for t in ts:
+        if t.dim() != 4:
+            raise ValueError("the Ulysses wrappers take dense [B][C][H][D] chunks (packed "
+                             "batches are not supported)")
+
+
 def check_split(Hq: int, Hkv: int, N: int) -> None:
     if Hq % N or Hkv % N:
         raise ValueError(f"Ulysses needs Hq ({Hq}) and Hkv ({Hkv}) divisible by the number "
@@ -96,6 +103,7 @@ class _UlyssesAttention(torch.autograd.Function):
     def forward(ctx, q, k, v, causal, scale, group, hooks):
         import torch.distributed as dist
         N = dist.get_world_size(group)
+        check_dense(q, k, v)
         check_split(q.shape[2], k.shape[2], N)
         tr = hooks.transpose
 
@@ -144,6 +152,7 @@ def ulysses_attention_single_device(q, k, v, world: int, causal: bool = True,
     from the full tensors (q [B][S][Hq][D], k/v [B][S][Hkv][D]): the same layout steps and
     per-head-group attention as ulysses_attention, with the all-to-alls done as plain
     copies.  Returns o, or (o, dq, dk, dv) when `do` is given."""
+    check_dense(q, k, v)
     hooks = (hooks or Hooks()).resolved()
     tr = hooks.transpose
     B, S = q.shape[0], q.shape[1]

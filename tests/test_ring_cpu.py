@@ -199,3 +199,14 @@ def test_gloo_ring_backward_equals_full_gradients(world, causal):
         assert p.exitcode == 0
     for r, errs in res:
         assert max(errs) < 1e-11, (r, errs)
+
+
+def test_wrappers_refuse_packed_layouts():
+    from long_context_attention_fwd_b200 import ulysses
+    packed = torch.zeros(64, 4, 8, dtype=torch.float64)
+    with pytest.raises(ValueError):
+        ring.ring_attn_fwd_single_device(packed, packed, packed, 2)
+    with pytest.raises(ValueError):
+        ring.ring_attn_bwd_single_device(packed, packed, packed, packed, None, packed, 2)
+    with pytest.raises(ValueError):
+        ulysses.ulysses_attention_single_device(packed, packed, packed, 2)
