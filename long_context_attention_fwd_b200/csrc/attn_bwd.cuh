@@ -57,6 +57,7 @@ struct Params {
   __nv_bfloat16* dv;
   int Hq, Hkv, G, T, causal;
   int ntile;              // tiles per head in the workspace = (T >> 7) + nseq
+  int group_major;        // CTA order: 1 = kv head outermost, 0 = kv head innermost
   float scale_log2;
   float scale;
   unsigned* status;
@@ -190,9 +191,26 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   const int lane = threadIdx.x & 31;
 
   // ---- work item: (sequence, kv head, 128-key tile); low tiles (most query tiles) first.
-  const int g = blockIdx.x % p.Hkv;
+  // Two orders of the same items.  Kv head innermost keeps the longest tiles of every
+  // group in the first wave.  Kv head outermost (dense batches only) keeps the CTAs
+  // resident at a time within one or two groups, so the dQ tiles they reduce into stay
+  // in L2 while the CTAs drift apart along the queries; the host takes it when one
+  // group's tiles fill a wave, so the longest tiles of later groups do not start late.
+  // Within a group of a dense batch the sequences are innermost (tile n of every
+  // sequence before tile n + 1); packed batches go sequence by sequence.
+  const unsigned nt = unsigned(p.ntile);
+  const int g = p.group_major ? int(blockIdx.x / nt) : int(blockIdx.x % unsigned(p.Hkv));
+  const int tix = p.group_major ? int(blockIdx.x % nt) : int(blockIdx.x / unsigned(p.Hkv));
   int seq, n, start, len;
-  if (!locate_block<7>(p.sv, int(blockIdx.x / p.Hkv), seq, n, start, len)) return;
+  if (p.sv.cu) {
+    if (!locate_block<7>(p.sv, tix, seq, n, start, len)) return;
+  } else {
+    seq = tix % p.sv.nseq;
+    n = tix / p.sv.nseq;
+    start = seq * p.sv.S;
+    len = p.sv.S;
+    if (n >= (len + 127) >> 7) return;
+  }
   const int nq = (len + 127) >> 7;
   const int m0 = p.causal ? n : 0;
   const int per_head = nq - m0;

@@ -454,6 +454,10 @@ attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o,
   p.T = int(T);
   p.causal = causal ? 1 : 0;
   p.ntile = w.ntile;
+  // Group-major CTA order once one kv head's tiles fill a wave of the GPU (measured on
+  // 28/4 heads, D = 128: 32K tokens 23.2 -> 22.4 ms; at 8K, 65 tiles a group, it would
+  // start the longest tiles of the last groups late: 1.51 -> 2.02 ms).
+  p.group_major = (!cu_seqlens && unsigned(w.ntile) >= dev->sms) ? 1 : 0;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.scale = scale;
   p.status = dev->status;
