@@ -408,23 +408,23 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       tc_fence_after();
       const float* lse_t = lse_s + st * 128 + cb;
       const float* dlt_t = delta_s + st * 128 + cb;
+      // The second 32 columns of S^T load while the first 32 are exponentiated.
       float pr[64];
-      {
-        uint32_t u0[32], u1[32];
-        tmem_ld32(tS + 0, u0);
-        tmem_ld32(tS + 32, u1);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          pr[i] = __uint_as_float(u0[i]);
-          pr[32 + i] = __uint_as_float(u1[i]);
-        }
-      }
+      uint32_t us[64];
+      auto half_s = [&](int hf) -> uint32_t(&)[32] {
+        return *reinterpret_cast<uint32_t(*)[32]>(us + 32 * hf);
+      };
+      tmem_ld32(tS + 0, half_s(0));
+      tmem_wait_ld_regs(half_s(0));
+      tmem_ld32(tS + 32, half_s(1));
       const bool diag = p.causal && m == n;
       const float4* lse4 = reinterpret_cast<const float4*>(lse_t);
       const uint64_t cc = f2_pack(c, c);
 #pragma unroll
       for (int i4 = 0; i4 < 16; ++i4) {
+        if (i4 == 8) tmem_wait_ld_regs(half_s(1));
+#pragma unroll
+        for (int u = 0; u < 4; ++u) pr[4 * i4 + u] = __uint_as_float(us[4 * i4 + u]);
         const float4 l4 = lse4[i4];
         float x0, x1, x2, x3;
         f2_unpack(f2_fma(f2_pack(pr[4 * i4], pr[4 * i4 + 1]), cc, f2_pack(-l4.x, -l4.y)), x0, x1);
@@ -456,15 +456,20 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                                        (it == 0 || mbar_wait(dq_full, (it - 1) & 1, wc, kSiteDqFull)));
       if (!ok) break;
       tc_fence_after();
+      // dP^T in two halves: the second loads while the first half's dS^T is computed.
+      // That half's TMEM store waits for the load, since warpgroup 1 stores dS^T over
+      // the columns of dP^T's second half.
       uint32_t u[64];
-      {
-        uint32_t* u0 = u;
-        tmem_ld32(tP + 0, *reinterpret_cast<uint32_t(*)[32]>(u0));
-        tmem_ld32(tP + 32, *reinterpret_cast<uint32_t(*)[32]>(u0 + 32));
-        tmem_wait_ld();
-      }
+      auto half_p = [&](int hf) -> uint32_t(&)[32] {
+        return *reinterpret_cast<uint32_t(*)[32]>(u + 32 * hf);
+      };
+      tmem_ld32(tP + 0, half_p(0));
+      tmem_wait_ld_regs(half_p(0));
+      tmem_ld32(tP + 32, half_p(1));
+      uint32_t pk_first[16];
 #pragma unroll
       for (int ch = 0; ch < 2; ++ch) {
+        if (ch == 1) tmem_wait_ld_regs(half_p(1));
         uint32_t pk[16];
         const float4* dl4 = reinterpret_cast<const float4*>(dlt_t + ch * 32);
 #pragma unroll
@@ -481,7 +486,13 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           pk[2 * i4] = pack_bf16x2(a0, a1);
           pk[2 * i4 + 1] = pack_bf16x2(a2, a3);
         }
-        tmem_st16(tDSst + ch * 16, pk);
+        if (ch == 0) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) pk_first[i] = pk[i];
+        } else {
+          tmem_st16(tDSst, pk_first);
+          tmem_st16(tDSst + 16, pk);
+        }
         // shared memory: this warpgroup's 64 query rows are 64-row block wg; local rows
         // ch*32 .. ch*32+31 are 16-byte chunks ch*4 .. ch*4+3 of the key row's line
 #pragma unroll
