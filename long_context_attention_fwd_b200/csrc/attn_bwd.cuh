@@ -10,7 +10,7 @@
 //     dS = P * (dP - Delta),  dV = P^T dO,  dK = scale dS^T Q,  dQ = scale dS K.
 //
 // Kernels:
-//   bwd_preprocess  Delta and LSE*log2(e) per query row into a tile-padded workspace
+//   bwd_preprocess  -Delta and -LSE*log2(e) per query row into a tile-padded workspace
 //                   (rows past a sequence end get LSE = +inf, so their P is exactly 0),
 //                   and zeroes the fp32 dQ accumulator rows.
 //   attn_bwd_kernel KV-stationary: one CTA holds a 128-key tile of one kv head (K, V in
@@ -51,8 +51,8 @@ constexpr int kSlab = 128 * 128;
 struct Params {
   SeqView sv;
   float* dq_acc;          // [Hq][ntile][D/4][128][4] fp32: one contiguous block per query tile
-  const float* lse2;      // [Hq][ntile][128]
-  const float* delta;     // [Hq][ntile][128]
+  const float* lse2;      // [Hq][ntile][128]: -LSE * log2(e) (negated: the P step adds it)
+  const float* delta;     // [Hq][ntile][128]: -Delta (negated: the dS step adds it)
   __nv_bfloat16* dk;      // [T][Hkv][D]
   __nv_bfloat16* dv;
   int Hq, Hkv, G, T, causal;
@@ -102,9 +102,10 @@ __host__ __device__ constexpr size_t dq_tile_offset(int r, int d) {
 
 // ---------------------------------------------------------------- preprocess
 // grid (ntile, Hq), 128 threads: one thread per query row of one 128-row tile.
-// Writes Delta_i = dO_i . O_i and LSE_i * log2(e) into the tile-padded workspace
-// (+inf / 0 for rows past the sequence end, so their probabilities are exactly 0)
-// and zeroes the tile's fp32 dQ block.
+// Writes -Delta_i = -(dO_i . O_i) and -LSE_i * log2(e) into the tile-padded workspace
+// (0 / -inf for rows past the sequence end, so their probabilities are exactly 0)
+// and zeroes the tile's fp32 dQ block.  Both are stored negated because the main
+// kernel adds them (one packed FMA / add, with no separate negation).
 template <int D>
 __global__ void __launch_bounds__(128)
 bwd_preprocess_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
@@ -140,8 +141,8 @@ bwd_preprocess_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* 
     l2 = lse[li] * 1.4426950408889634f;
   }
   const size_t wi = (size_t(h) * ntile + blockIdx.x) * 128 + r;
-  lse2[wi] = l2;
-  delta[wi] = dl;
+  lse2[wi] = -l2;
+  delta[wi] = -dl;
   float4* z = reinterpret_cast<float4*>(dq_acc + (size_t(h) * ntile + blockIdx.x) * 128 * D);
 #pragma unroll 4
   for (int i = 0; i < D / 4; ++i) z[i * 128 + r] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -420,23 +421,30 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const bool diag = p.causal && m == n;
       const float4* lse4 = reinterpret_cast<const float4*>(lse_t);
       const uint64_t cc = f2_pack(c, c);
+      // Only the diagonal tile (causal) and keys past a sequence's end (full mask) need
+      // the per-element select; every other tile takes the unmasked path.
+      const bool masked = diag || !key_ok;
+      auto p_quads = [&](int i4_0, bool msk) {
 #pragma unroll
-      for (int i4 = 0; i4 < 16; ++i4) {
-        if (i4 == 8) tmem_wait_ld_regs(half_s(1));
+        for (int i4 = i4_0; i4 < i4_0 + 8; ++i4) {
 #pragma unroll
-        for (int u = 0; u < 4; ++u) pr[4 * i4 + u] = __uint_as_float(us[4 * i4 + u]);
-        const float4 l4 = lse4[i4];
-        float x0, x1, x2, x3;
-        f2_unpack(f2_fma(f2_pack(pr[4 * i4], pr[4 * i4 + 1]), cc, f2_pack(-l4.x, -l4.y)), x0, x1);
-        f2_unpack(f2_fma(f2_pack(pr[4 * i4 + 2], pr[4 * i4 + 3]), cc, f2_pack(-l4.z, -l4.w)), x2, x3);
-        const float xv[4] = {x0, x1, x2, x3};
+          for (int u = 0; u < 4; ++u) pr[4 * i4 + u] = __uint_as_float(us[4 * i4 + u]);
+          const float4 l4 = lse4[i4];
+          float x0, x1, x2, x3;
+          f2_unpack(f2_fma(f2_pack(pr[4 * i4], pr[4 * i4 + 1]), cc, f2_pack(l4.x, l4.y)), x0, x1);
+          f2_unpack(f2_fma(f2_pack(pr[4 * i4 + 2], pr[4 * i4 + 3]), cc, f2_pack(l4.z, l4.w)), x2, x3);
+          const float xv[4] = {x0, x1, x2, x3};
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int i = 4 * i4 + u;
-          const float e = ex2_approx(xv[u]);
-          pr[i] = (key_ok && !(diag && cb + i < r)) ? e : 0.f;
+          for (int u = 0; u < 4; ++u) {
+            const int i = 4 * i4 + u;
+            const float e = ex2_approx(xv[u]);
+            pr[i] = msk ? ((key_ok && !(diag && cb + i < r)) ? e : 0.f) : e;
+          }
         }
-      }
+      };
+      if (masked) p_quads(0, true); else p_quads(0, false);
+      tmem_wait_ld_regs(half_s(1));
+      if (masked) p_quads(8, true); else p_quads(8, false);
 #pragma unroll
       for (int ch = 0; ch < 2; ++ch) {
         uint32_t pk[16];
@@ -479,10 +487,10 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           float a0, a1, a2, a3;
           f2_unpack(f2_mul(f2_pack(pr[c0], pr[c0 + 1]),
                            f2_add(f2_pack(__uint_as_float(u[c0]), __uint_as_float(u[c0 + 1])),
-                                  f2_pack(-d4.x, -d4.y))), a0, a1);
+                                  f2_pack(d4.x, d4.y))), a0, a1);
           f2_unpack(f2_mul(f2_pack(pr[c0 + 2], pr[c0 + 3]),
                            f2_add(f2_pack(__uint_as_float(u[c0 + 2]), __uint_as_float(u[c0 + 3])),
-                                  f2_pack(-d4.z, -d4.w))), a2, a3);
+                                  f2_pack(d4.z, d4.w))), a2, a3);
           pk[2 * i4] = pack_bf16x2(a0, a1);
           pk[2 * i4 + 1] = pack_bf16x2(a2, a3);
         }
