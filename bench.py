@@ -116,10 +116,51 @@ def measured_traffic(workload: str, kernel: str):
 
 
 # ---------------------------------------------------------------- clocks
+CLOCK_FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+CLOCK_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+
+def summarize_clocks(lines, t0: float, t1: float) -> dict:
+    """Summary of `nvidia-smi --query-gpu=CLOCK_FIELDS --format=csv,noheader,nounits` lines
+    for the samples taken in the wall-clock window [t0, t1] (seconds since the epoch):
+    median SM clock, the maximum SM clock, every throttle reason seen active and the
+    sample count.  When no sample falls in the window (a region shorter than the sampling
+    interval) the samples just around it are used, and `window` says so."""
+    import datetime
+    rows = []
+    for line in lines:
+        parts = [x.strip() for x in line.split(",")]
+        if len(parts) < 10:
+            continue
+        try:
+            ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+            rows.append((ts, float(parts[2]), float(parts[3]), float(parts[4]), parts[5:]))
+        except ValueError:
+            continue
+    if not rows:
+        return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+    inside = [r for r in rows if t0 <= r[0] <= t1]
+    window = "timed region"
+    if not inside:
+        near = sorted(rows, key=lambda r: min(abs(r[0] - t0), abs(r[0] - t1)))
+        inside = near[:2]
+        window = "nearest samples (none inside the timed region)"
+    reasons = set()
+    for r in inside:
+        for n, v in zip(CLOCK_REASONS, r[4][1:]):
+            if v.lower().startswith("active"):
+                reasons.add(n)
+    return {"sm_mhz": statistics.median(r[1] for r in inside),
+            "sm_max_mhz": max(r[2] for r in rows),
+            "reasons": sorted(reasons), "samples": len(inside),
+            "power_w_max": max(r[3] for r in inside), "window": window}
+
+
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """nvidia-smi every 50 ms into gpurun_out/clocks_bench_<pid>.csv, summarised over the
+    timed region's wall-clock window."""
 
     def __init__(self, index: int):
         self.index = index
@@ -131,43 +172,24 @@ class ClockSampler:
             os.makedirs(os.path.dirname(self.path), exist_ok=True)
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={CLOCK_FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"], stdout=self.f,
                 stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
 
-    def stop(self) -> dict:
+    def stop(self, t0: float, t1: float) -> dict:
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.1)  # the sample after the region's end
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
         except Exception:
             self.proc.kill()
         self.f.close()
-        rows = []
-        for line in open(self.path):
-            parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[4:]))
-            except ValueError:
-                continue
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = set()
-        for r in rows:
-            for n, v in zip(names, r[3][1:]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        loaded = [r for r in rows if r[2] > 300.0] or rows
-        return {"sm_mhz": statistics.median(r[0] for r in loaded),
-                "sm_max_mhz": max(r[1] for r in rows),
-                "reasons": sorted(reasons), "samples": len(rows),
-                "power_w_max": max(r[2] for r in rows)}
+        with open(self.path) as f:
+            return summarize_clocks(f.readlines(), t0, t1)
 
 
 # ---------------------------------------------------------------- CPU oracle
@@ -510,12 +532,14 @@ def run_gpu(args, w: I.Workload):
     sampler.start()
     time.sleep(0.3)
     barrier()
+    wall0 = time.time()
     t_start.record(stream)
     for i in range(args.steps):
         step(evs[i])
     t_end.record(stream)
     barrier()
-    clocks = sampler.stop()
+    wall1 = time.time()
+    clocks = sampler.stop(wall0, wall1)
     total_ms = t_start.elapsed_time(t_end)
     fwd_ms = [e[0].elapsed_time(e[1]) for e in evs]
     bwd_ms = [e[1].elapsed_time(e[2]) for e in evs]

@@ -33,3 +33,37 @@ def test_reference_arm_line_has_the_contract_keys():
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}
+
+
+def test_clock_summary_keeps_the_timed_window_only():
+    """The bench's clock record: samples outside the timed region (the idle lead-in, the
+    work after it) change neither the median clock nor the throttle reasons."""
+    import datetime
+    import bench
+
+    base = datetime.datetime(2026, 12, 2, 12, 0, 0)
+
+    def line(dt_ms, sm, power, hw="Not Active", cap="Not Active"):
+        ts = (base + datetime.timedelta(milliseconds=dt_ms)).strftime("%Y/%m/%d %H:%M:%S.%f")[:-3]
+        return f"{ts}, 0, {sm}, 1965, {power}, 0x0, {hw}, Not Active, Not Active, {cap}\n"
+
+    lines = [line(0, 345, 120.0, hw="Active"),         # idle lead-in, outside the window
+             line(100, 1800, 700.0, cap="Active"),
+             line(150, 1900, 720.0),
+             line(200, 1850, 710.0),
+             "garbage line\n",
+             line(400, 1965, 150.0, hw="Active")]       # after the window
+    t0 = (base + datetime.timedelta(milliseconds=90)).timestamp()
+    t1 = (base + datetime.timedelta(milliseconds=210)).timestamp()
+    c = bench.summarize_clocks(lines, t0, t1)
+    assert c["samples"] == 3 and c["window"] == "timed region"
+    assert c["sm_mhz"] == 1850.0 and c["sm_max_mhz"] == 1965.0
+    assert c["reasons"] == ["sw_power_cap"]
+    assert c["power_w_max"] == 720.0
+
+    # a region shorter than the sampling interval: the nearest samples stand in, labelled
+    t0 = (base + datetime.timedelta(milliseconds=120)).timestamp()
+    t1 = (base + datetime.timedelta(milliseconds=130)).timestamp()
+    c = bench.summarize_clocks(lines, t0, t1)
+    assert c["samples"] == 2 and c["window"].startswith("nearest")
+    assert bench.summarize_clocks(["nothing parseable\n"], t0, t1)["samples"] == 0
