@@ -159,13 +159,16 @@ def summarize_clocks(lines, t0: float, t1: float) -> dict:
 
 
 class ClockSampler:
-    """nvidia-smi every 50 ms into gpurun_out/clocks_bench_<pid>.csv, summarised over the
-    timed region's wall-clock window."""
+    """nvidia-smi every 50 ms into clocks_bench_<pid>.csv, summarised over the timed
+    region's wall-clock window.  The log goes to $ATTN_BENCH_CLOCKS_DIR when set, else to
+    the system's temporary directory."""
 
     def __init__(self, index: int):
+        import tempfile
         self.index = index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_bench_{os.getpid()}.csv")
+        folder = os.environ.get("ATTN_BENCH_CLOCKS_DIR") or tempfile.gettempdir()
+        self.path = os.path.join(folder, f"clocks_bench_{os.getpid()}.csv")
 
     def start(self):
         try:

@@ -71,7 +71,7 @@ def make_case(B, Hq, Hkv, S, D, causal=True, lens=None, seed=1234, qkv_mult=0.5,
     return w
 
 
-class GpuRun:
+class DeviceRun:
     """Runs attn_fwd / attn_bwd of the library on a workload's seeded inputs."""
 
     def __init__(self, w: I.Workload, device="cuda", poison=True):

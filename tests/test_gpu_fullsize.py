@@ -15,7 +15,7 @@ import numpy as np
 import pytest
 
 import oracle
-from helpers import (TOL_GRAD, TOL_LSE, GpuRun, o_error_report, oracle_args, rel_l2)
+from helpers import (TOL_GRAD, TOL_LSE, DeviceRun, o_error_report, oracle_args, rel_l2)
 from long_context_attention_fwd_b200 import inputs as I
 
 torch = pytest.importorskip("torch")
@@ -40,7 +40,7 @@ def _sample_rows(w, rng, n_random=24):
 @pytest.mark.parametrize("idx", [1, 2, 3, 4], ids=["S8K", "S32K", "varlen32K", "mha_D64_outliers"])
 def test_full_size_sampled(idx):
     w = I.workload(idx)
-    run = GpuRun(w, poison=False)
+    run = DeviceRun(w, poison=False)
     g = run.np_out()
     q, k, v, do, kw = oracle_args(w, run.x)
     rng = np.random.default_rng(100 + idx)

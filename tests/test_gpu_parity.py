@@ -9,7 +9,7 @@ import numpy as np
 import pytest
 
 import oracle
-from helpers import (TOL_GRAD, TOL_LSE, GpuRun, make_case, o_error_report, oracle_args, rel_l2)
+from helpers import (TOL_GRAD, TOL_LSE, DeviceRun, make_case, o_error_report, oracle_args, rel_l2)
 from long_context_attention_fwd_b200 import inputs as I
 
 torch = pytest.importorskip("torch")
@@ -43,7 +43,7 @@ def _ref(w, x):
 @pytest.mark.gpu
 @pytest.mark.parametrize("name,w", SMALL, ids=[c[0] for c in SMALL])
 def test_small_elementwise(name, w):
-    run = GpuRun(w)
+    run = DeviceRun(w)
     g = run.np_out()
     r = _ref(w, run.x)
     rep = o_error_report(g["o"], r["o"], r["o_absv"])
@@ -61,8 +61,8 @@ def test_small_elementwise(name, w):
 @pytest.mark.gpu
 def test_forward_and_dkdv_are_deterministic():
     w = make_case(1, 4, 2, 700, 128, True, seed=21)
-    a = GpuRun(w)
-    b = GpuRun(w)
+    a = DeviceRun(w)
+    b = DeviceRun(w)
     for t in ("o", "lse", "dk", "dv"):
         assert torch.equal(getattr(a, t), getattr(b, t)), t
     torch.testing.assert_close(a.dq.float(), b.dq.float(), rtol=0, atol=2e-2)
@@ -72,7 +72,7 @@ def test_forward_and_dkdv_are_deterministic():
 def test_packed_equals_separate_on_gpu():
     lens = [300, 1, 0, 257, 128]
     w = make_case(0, 4, 1, 0, 128, True, seed=22, lens=lens)
-    packed = GpuRun(w)
+    packed = DeviceRun(w)
     cu = np.concatenate([[0], np.cumsum(lens)])
     from long_context_attention_fwd_b200 import ops
     for s, L in enumerate(lens):
@@ -96,7 +96,7 @@ def test_packed_equals_separate_on_gpu():
 def test_autograd_wrapper_matches_explicit_calls():
     from long_context_attention_fwd_b200 import ops
     w = make_case(1, 2, 1, 256, 64, True, seed=23)
-    run = GpuRun(w)
+    run = DeviceRun(w)
     q = run.q.clone().requires_grad_(True)
     k = run.k.clone().requires_grad_(True)
     v = run.v.clone().requires_grad_(True)

@@ -13,7 +13,7 @@ import numpy as np
 import pytest
 
 import oracle
-from helpers import TOL_GRAD, TOL_LSE, GpuRun, make_case, o_error_report, rel_l2
+from helpers import TOL_GRAD, TOL_LSE, DeviceRun, make_case, o_error_report, rel_l2
 from long_context_attention_fwd_b200 import inputs as I
 
 torch = pytest.importorskip("torch")
@@ -38,7 +38,7 @@ def test_backward_orders(name, w, group_major):
     G = w.Hq // w.Hkv
     ntile = (w.B * w.S >> 7) + w.B
     assert (ntile >= 148) == group_major, "case no longer lands on its side of the threshold"
-    run = GpuRun(w)
+    run = DeviceRun(w)
     g = run.np_out()
     q, k, v, do = (I.bf16_bits_to_f64(run.x[n]) for n in ("q", "k", "v", "do"))
     # first, middle and last sequence; first and last kv head
