@@ -19,7 +19,7 @@ rank after rank on this GPU; and "decode": attention of one new token per sequen
 a 32K-token KV cache (HBM-bound); and "fp8_fwd": the e4m3 forward on the bench workload.
 All are measured after the timed steps.
 
---impl reference times the fp64 CPU oracle (the reference arm of this build) on a
+--impl reference times the fp64 CPU oracle (the bench's reference arm) on a
 bounded sample of the same workload: the first tokens of the causal sequence form
 an exact sub-problem, so each step runs the oracle's forward and backward on them.
 """

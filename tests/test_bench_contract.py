@@ -1,5 +1,5 @@
 """The bench line's contract, checked on the CPU through the reference arm (the fp64
-oracle on a bounded sample): one JSON line with the keys the driver reads, the same
+oracle on a bounded sample): one JSON line with every key of the bench contract, the same
 metric and workload as the GPU arm, and the reference-arm extras (impl, cpu_baseline,
 an e2e object with zero host<->device bytes)."""
 import json
