@@ -271,6 +271,50 @@ def test_matches_torch_sdpa_fp64(causal, gqa):
     np.testing.assert_allclose(lse[0], torch.logsumexp(s, -1).numpy(), atol=1e-12)
 
 
+# ---------------------------------------------------------------- brute force
+def _brute_force_long_double(q, k, v, causal, scale, B, S):
+    """The definition written out element by element in extended precision
+    (np.longdouble), with no maximum subtracted before exponentiating:
+    O_i = sum_j exp(s_ij) v_j / sum_j exp(s_ij), LSE_i = ln sum_j exp(s_ij), over the keys
+    j the mask lets row i see, s_ij = scale * q_i . k_j, query head h reading kv head
+    h // (Hq / Hkv)."""
+    T, Hq, D = q.shape
+    Hkv = k.shape[1]
+    G = Hq // Hkv
+    ld = np.longdouble
+    o = np.zeros((T, Hq, D), dtype=ld)
+    lse = np.zeros((B, Hq, S), dtype=ld)
+    for b in range(B):
+        for h in range(Hq):
+            g = h // G
+            for i in range(S):
+                ti = b * S + i
+                den = ld(0)
+                num = np.zeros(D, dtype=ld)
+                for j in range(S if not causal else i + 1):
+                    tj = b * S + j
+                    s = ld(scale) * sum(ld(q[ti, h, d]) * ld(k[tj, g, d]) for d in range(D))
+                    e = np.exp(s)
+                    den += e
+                    num += e * v[tj, g].astype(ld)
+                o[ti, h] = num / den
+                lse[b, h, i] = np.log(den)
+    return o, lse
+
+
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("shape", [(1, 4, 4, 32, 8), (2, 6, 2, 13, 3)],
+                         ids=["B1_mha4_S32_D8", "B2_gqa6x2_S13_D3"])
+def test_brute_force_long_double(causal, shape):
+    B, Hq, Hkv, S, D = shape
+    scale = 0.37
+    q, k, v = rnd((B * S, Hq, D), 51), rnd((B * S, Hkv, D), 52), rnd((B * S, Hkv, D), 53)
+    o, lse = oracle.fwd(q, k, v, causal, scale, B=B, S=S)
+    o_bf, lse_bf = _brute_force_long_double(q, k, v, causal, scale, B, S)
+    assert np.abs(o - o_bf.astype(np.float64)).max() <= 1e-12
+    assert np.abs(lse - lse_bf.astype(np.float64)).max() <= 1e-12
+
+
 # ---------------------------------------------------------------- row APIs
 def test_row_apis_agree_with_full():
     lens = [70, 3, 45]
