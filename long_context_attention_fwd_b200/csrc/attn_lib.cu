@@ -66,6 +66,57 @@ std::mutex g_mu;
 DeviceState g_dev[kMaxDevices];
 EncodeTiledFn g_encode = nullptr;
 
+// The calling thread's current device.  Entry points make the device that owns their
+// tensors current (launches and kernel attributes need it) and give the caller's choice
+// back when they return.  The previous device is only made current again when its
+// primary context is already active: cudaSetDevice would otherwise create a context,
+// and take its memory, on a device this process never used.
+typedef CUresult (*DeviceGetFn)(CUdevice*, int);
+typedef CUresult (*PrimaryCtxStateFn)(CUdevice, unsigned int*, int*);
+std::once_flag g_ctx_fns_once;
+DeviceGetFn g_device_get = nullptr;
+PrimaryCtxStateFn g_primary_ctx_state = nullptr;
+
+bool primary_context_active(int ordinal) {
+  std::call_once(g_ctx_fns_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuDeviceGet", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_device_get = reinterpret_cast<DeviceGetFn>(fn);
+    fn = nullptr;
+    if (cudaGetDriverEntryPoint("cuDevicePrimaryCtxGetState", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_primary_ctx_state = reinterpret_cast<PrimaryCtxStateFn>(fn);
+    (void)cudaGetLastError();
+  });
+  if (!g_device_get || !g_primary_ctx_state) return false;
+  CUdevice d;
+  if (g_device_get(&d, ordinal) != CUDA_SUCCESS) return false;
+  unsigned flags = 0;
+  int active = 0;
+  return g_primary_ctx_state(d, &flags, &active) == CUDA_SUCCESS && active != 0;
+}
+
+struct DeviceRestore {
+  int prev = -1;
+  DeviceRestore() {
+    if (cudaGetDevice(&prev) != cudaSuccess) {
+      prev = -1;
+      (void)cudaGetLastError();
+    }
+  }
+  ~DeviceRestore() {
+    int cur = -1;
+    if (prev < 0 || cudaGetDevice(&cur) != cudaSuccess || cur == prev) return;
+    if (primary_context_active(prev) && cudaSetDevice(prev) != cudaSuccess)
+      (void)cudaGetLastError();  // leave no stale error for the caller's next check
+  }
+  DeviceRestore(const DeviceRestore&) = delete;
+  DeviceRestore& operator=(const DeviceRestore&) = delete;
+};
+
 // Per-device set-up (once): capability check, status-word address, kernel attributes.
 // `ptr` (optional) is a device pointer of the call: its device is made current on the
 // calling thread first, so that a call from any host thread (autograd's worker thread,
@@ -320,6 +371,7 @@ attn_status attn_check_cu_seqlens(const int32_t* cu, int B, int S) {
 attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                      int Hq, int Hkv, int S, int D, int causal, float scale,
                      const int32_t* cu_seqlens, void* stream) {
+  DeviceRestore restore_device;
   long long T = 0;
   attn_status st = check_sizes(B, Hq, Hkv, S, D, scale, cu_seqlens != nullptr, &T);
   if (st != ATTN_OK) return st;
@@ -359,6 +411,7 @@ attn_status attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, f
                          int Hq, int Hkv, int S, int D, int causal, float scale, float q_descale,
                          float k_descale, float v_descale, const int32_t* cu_seqlens,
                          void* stream) {
+  DeviceRestore restore_device;
   long long T = 0;
   attn_status st = check_sizes(B, Hq, Hkv, S, D, scale, cu_seqlens != nullptr, &T);
   if (st != ATTN_OK) return st;
@@ -405,6 +458,7 @@ attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o,
                      int Hq, int Hkv, int S, int D, int causal, float scale,
                      const int32_t* cu_seqlens, void* workspace, size_t workspace_bytes,
                      void* stream) {
+  DeviceRestore restore_device;
   long long T = 0;
   attn_status st = check_sizes(B, Hq, Hkv, S, D, scale, cu_seqlens != nullptr, &T);
   if (st != ATTN_OK) return st;
@@ -480,6 +534,7 @@ attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o,
 
 attn_status attn_merge(const void* const* o_parts, const float* const* lse_parts, int nparts,
                        void* o, float* lse, int B, int H, int S, int D, void* stream) {
+  DeviceRestore restore_device;
   if (nparts < 1 || nparts > ATTN_MERGE_MAX_PARTS || !o_parts || !lse_parts || !o || !lse)
     return ATTN_ERR_INVALID_ARG;
   if (B < 1 || H < 1 || S < 1) return ATTN_ERR_INVALID_ARG;
@@ -539,6 +594,7 @@ attn_status attn_decode(const void* q, const void* k_cache, const void* v_cache,
                         const int32_t* cache_len, void* o, float* lse, int B, int Hq, int Hkv,
                         int Lmax, int D, float scale, void* workspace, size_t workspace_bytes,
                         void* stream) {
+  DeviceRestore restore_device;
   attn_status st = check_decode_sizes(B, Hq, Hkv, Lmax, D, scale);
   if (st != ATTN_OK) return st;
   if (!q || !k_cache || !v_cache || !cache_len || !o || !lse || !workspace)
@@ -606,6 +662,7 @@ attn_status attn_decode(const void* q, const void* k_cache, const void* v_cache,
 }
 
 attn_status attn_accumulate_bf16(float* acc, const void* x, long long n, int init, void* stream) {
+  DeviceRestore restore_device;
   if (!acc || !x || n < 1) return ATTN_ERR_INVALID_ARG;
   if (n % 8) return ATTN_ERR_INVALID_ARG;
   if (!aligned(acc, 16) || !aligned(x, 16)) return ATTN_ERR_MISALIGNED;
@@ -622,6 +679,7 @@ attn_status attn_accumulate_bf16(float* acc, const void* x, long long n, int ini
 }
 
 attn_status attn_convert_f32_bf16(void* out, const float* in, long long n, void* stream) {
+  DeviceRestore restore_device;
   if (!out || !in || n < 1) return ATTN_ERR_INVALID_ARG;
   if (n % 8) return ATTN_ERR_INVALID_ARG;
   if (!aligned(out, 16) || !aligned(in, 16)) return ATTN_ERR_MISALIGNED;
@@ -639,6 +697,7 @@ attn_status attn_convert_f32_bf16(void* out, const float* in, long long n, void*
 
 attn_status attn_transpose_blocks(const void* in, void* out, long long n_outer, long long n_inner,
                                   long long block_bytes, void* stream) {
+  DeviceRestore restore_device;
   if (!in || !out || n_outer < 1 || n_inner < 1 || block_bytes < 16) return ATTN_ERR_INVALID_ARG;
   if (block_bytes % 16) return ATTN_ERR_MISALIGNED;
   if (!aligned(in, 16) || !aligned(out, 16)) return ATTN_ERR_MISALIGNED;
@@ -714,6 +773,7 @@ extern "C" attn_status attn_selftest_wait_timeout(unsigned long long timeout_ns,
 extern "C" attn_status attn_selftest_umma(int mode, int D, const void* a, const void* b,
                                           const float* pin, const void* at, float* c,
                                           void* stream) {
+  DeviceRestore restore_device;
   if (mode < 0 || mode > 2) return ATTN_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
   if (!b || !c || (mode == 0 && !a) || (mode == 1 && !pin) || (mode == 2 && !at))
@@ -739,6 +799,7 @@ extern "C" attn_status attn_selftest_umma(int mode, int D, const void* a, const 
 
 extern "C" attn_status attn_selftest_umma_fp8(int mode, const void* a, const void* b,
                                               const float* pin, float* pq, float* c, void* stream) {
+  DeviceRestore restore_device;
   if (mode != 3 && mode != 4) return ATTN_ERR_INVALID_ARG;
   if (!b || !c || (mode == 3 && !a) || (mode == 4 && (!pin || !pq))) return ATTN_ERR_INVALID_ARG;
   if (!aligned(b, 16) || (a && !aligned(a, 16)) || (pin && !aligned(pin, 16)) ||
@@ -774,6 +835,7 @@ extern "C" attn_status attn_bwd_noalloc(const void* q, const void* k, const void
                                         void* dq, void* dk, void* dv, int B, int Hq, int Hkv,
                                         int S, int D, int causal, float scale,
                                         const int32_t* cu_seqlens, void* stream) {
+  DeviceRestore restore_device;
   const size_t need = attn_bwd_workspace_size(B, Hq, S, D, cu_seqlens);
   if (need == 0) return ATTN_ERR_INVALID_ARG;  // the same size checks attn_bwd applies
   if (need > size_t(ATTN_BWD_NOALLOC_MAX_BYTES)) {

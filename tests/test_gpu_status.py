@@ -66,3 +66,24 @@ def test_calls_from_another_host_thread():
     t.join()
     assert "e" not in box, box.get("e")
     assert torch.equal(box["r"][1], ref[1]) and torch.equal(box["r"][2], ref[2])
+
+
+@pytest.mark.gpu
+def test_calls_leave_the_callers_current_device_alone():
+    """Each entry point makes the tensors' device current for its own launches and gives
+    the calling thread its current device back on return."""
+    if torch.cuda.device_count() < 2:
+        pytest.skip("needs two GPUs")
+    from long_context_attention_fwd_b200 import ops
+    torch.cuda.set_device(0)
+    torch.zeros(1, device="cuda:0")  # device 0's context is active
+    q = torch.randn(1, 256, 2, 64, device="cuda:1").bfloat16()
+    o, lse = ops.attn_fwd(q, q, q, causal=True)
+    assert torch.cuda.current_device() == 0
+    dq, dk, dv = ops.attn_bwd(q, q, q, o, lse, torch.ones_like(q))
+    assert torch.cuda.current_device() == 0
+    torch.cuda.synchronize(1)
+    with torch.cuda.device(1):
+        o1, _ = ops.attn_fwd(q, q, q, causal=True)
+    torch.cuda.synchronize(1)
+    assert torch.equal(o, o1)
