@@ -27,7 +27,11 @@ def _stream(device) -> int:
     return torch.cuda.current_stream(device).cuda_stream
 
 
-def _dims(q: torch.Tensor, k: torch.Tensor, cu_seqlens: Optional[torch.Tensor]):
+def _dims(q: torch.Tensor, k: torch.Tensor, cu_seqlens: Optional[torch.Tensor],
+          v: Optional[torch.Tensor] = None):
+    _same_device(q.device, k, v, cu_seqlens)
+    if v is not None and v.shape != k.shape:
+        raise ValueError("v must have k's shape")
     if cu_seqlens is None:
         if q.dim() != 4 or k.dim() != 4:
             raise ValueError("dense inputs must be [B, S, H, D]")
@@ -41,11 +45,40 @@ def _dims(q: torch.Tensor, k: torch.Tensor, cu_seqlens: Optional[torch.Tensor]):
         S, Hq, D = q.shape
         Hkv = k.shape[1]
         B = cu_seqlens.numel() - 1
-        if cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_cuda:
-            raise ValueError("cu_seqlens must be an int32 CUDA tensor")
+        if cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_cuda \
+                or not cu_seqlens.is_contiguous() or cu_seqlens.dim() != 1:
+            raise ValueError("cu_seqlens must be a contiguous 1-D int32 CUDA tensor")
         if k.shape[0] != S or k.shape[2] != D:
             raise ValueError("k/v shape does not match q")
     return B, S, Hq, Hkv, D
+
+
+def _same_device(device, *ts) -> None:
+    for t in ts:
+        if t is not None and t.device != device:
+            raise ValueError(f"all tensors must be on {device} (one is on {t.device})")
+
+
+def _check_tensor(t: Optional[torch.Tensor], name: str, shape, dtype, device) -> None:
+    """A caller-supplied output, or an input whose size the kernel takes from another
+    tensor, must be exactly what the kernel writes or reads: a smaller one would send
+    the kernel past its end."""
+    if t is None:
+        return
+    if tuple(t.shape) != tuple(shape) or t.dtype != dtype or t.device != device \
+            or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous {dtype} tensor of shape "
+                         f"{tuple(shape)} on {device}")
+
+
+def _workspace_bytes(ws: torch.Tensor, device) -> int:
+    if not ws.is_cuda or ws.device != device or not ws.is_contiguous():
+        raise ValueError(f"workspace must be a contiguous tensor on {device}")
+    return ws.numel() * ws.element_size()
+
+
+def _lse_shape(B: int, S: int, Hq: int, packed: bool):
+    return (Hq, S) if packed else (B, Hq, S)
 
 
 def _check_inputs(*ts: torch.Tensor) -> None:
@@ -64,13 +97,15 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = T
              lse: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
     """Fused forward: returns (o, lse); lse is fp32 [B,Hq,S] (dense) or [Hq,T] (packed)."""
     _check_inputs(q, k, v)
-    B, S, Hq, Hkv, D = _dims(q, k, cu_seqlens)
+    B, S, Hq, Hkv, D = _dims(q, k, cu_seqlens, v)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
+    shape = _lse_shape(B, S, Hq, cu_seqlens is not None)
+    _check_tensor(out, "out", q.shape, torch.bfloat16, q.device)
+    _check_tensor(lse, "lse", shape, torch.float32, q.device)
     if out is None:
         out = torch.empty_like(q)
     if lse is None:
-        shape = (Hq, S) if cu_seqlens is not None else (B, Hq, S)
         lse = torch.empty(shape, dtype=torch.float32, device=q.device)
     st = capi.attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
                        B, Hq, Hkv, S, D, causal, scale,
@@ -93,20 +128,28 @@ def attn_bwd(q, k, v, o, lse, dout, causal: bool = True, scale: Optional[float] 
              workspace: Optional[torch.Tensor] = None):
     """Fused backward: returns (dq, dk, dv)."""
     _check_inputs(q, k, v, o, dout)
-    B, S, Hq, Hkv, D = _dims(q, k, cu_seqlens)
+    B, S, Hq, Hkv, D = _dims(q, k, cu_seqlens, v)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
+    dev = q.device
+    _check_tensor(o, "o", q.shape, torch.bfloat16, dev)
+    _check_tensor(dout, "dout", q.shape, torch.bfloat16, dev)
+    _check_tensor(lse, "lse", _lse_shape(B, S, Hq, cu_seqlens is not None), torch.float32, dev)
+    _check_tensor(dq, "dq", q.shape, torch.bfloat16, dev)
+    _check_tensor(dk, "dk", k.shape, torch.bfloat16, dev)
+    _check_tensor(dv, "dv", v.shape, torch.bfloat16, dev)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
     need = attn_bwd_workspace_size(q, cu_seqlens)
     if workspace is None:
-        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_bytes = _workspace_bytes(workspace, dev)
     st = capi.attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
                        dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
                        B, Hq, Hkv, S, D, causal, scale,
                        cu_seqlens.data_ptr() if cu_seqlens is not None else None,
-                       workspace.data_ptr(), workspace.numel(), _stream(q.device))
+                       workspace.data_ptr(), ws_bytes, _stream(q.device))
     capi.check(st, "attn_bwd")
     return dq, dk, dv
 
@@ -166,6 +209,8 @@ def attn_merge(o_parts: Sequence[torch.Tensor], lse_parts: Sequence[torch.Tensor
         groups = [attn_merge(o_parts[i:i + MERGE_MAX_PARTS], lse_parts[i:i + MERGE_MAX_PARTS])
                   for i in range(0, len(o_parts), MERGE_MAX_PARTS)]
         return attn_merge([g[0] for g in groups], [g[1] for g in groups], out, lse)
+    _check_tensor(out, "out", o0.shape, torch.bfloat16, o0.device)
+    _check_tensor(lse, "lse", lse_shape, torch.float32, o0.device)
     out = torch.empty_like(o0) if out is None else out
     lse = torch.empty_like(l0) if lse is None else lse
     st = capi.attn_merge([t.data_ptr() for t in o_parts], [t.data_ptr() for t in lse_parts],
@@ -187,8 +232,9 @@ def transpose_blocks(x: torch.Tensor, n_outer: int, n_inner: int,
     blk = n // (n_outer * n_inner)
     if out is None:
         out = torch.empty((n_inner, n_outer, blk), dtype=x.dtype, device=x.device)
-    elif out.numel() != n or not out.is_contiguous() or out.dtype != x.dtype:
-        raise ValueError("out must be contiguous, of x's dtype and size")
+    elif out.numel() != n or not out.is_contiguous() or out.dtype != x.dtype \
+            or out.device != x.device:
+        raise ValueError("out must be contiguous, of x's dtype and size, on x's device")
     st = capi.attn_transpose_blocks(x.data_ptr(), out.data_ptr(), n_outer, n_inner,
                                     blk * x.element_size(), _stream(x.device))
     capi.check(st, "attn_transpose_blocks")
@@ -214,18 +260,23 @@ def attn_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
     Bk, Lmax, Hkv, Dk = k_cache.shape
     if Bk != B or Dk != D:
         raise ValueError("cache shape does not match q")
-    if cache_len.dtype != torch.int32 or not cache_len.is_cuda or cache_len.numel() != B:
-        raise ValueError("cache_len must be an int32 CUDA tensor of B entries")
+    if cache_len.dtype != torch.int32 or not cache_len.is_cuda or cache_len.numel() != B \
+            or not cache_len.is_contiguous():
+        raise ValueError("cache_len must be a contiguous int32 CUDA tensor of B entries")
+    _same_device(q.device, k_cache, v_cache, cache_len)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
+    _check_tensor(out, "out", q.shape, torch.bfloat16, q.device)
+    _check_tensor(lse, "lse", (B, Hq), torch.float32, q.device)
     out = torch.empty_like(q) if out is None else out
     lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device) if lse is None else lse
     need = capi.attn_decode_workspace_size(B, Hq, Hkv, Lmax, D)
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    ws_bytes = _workspace_bytes(workspace, q.device)
     st = capi.attn_decode(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
                           cache_len.data_ptr(), out.data_ptr(), lse.data_ptr(), B, Hq, Hkv, Lmax,
-                          D, scale, workspace.data_ptr(), workspace.numel(), _stream(q.device))
+                          D, scale, workspace.data_ptr(), ws_bytes, _stream(q.device))
     capi.check(st, "attn_decode")
     return out, lse
 
@@ -248,13 +299,15 @@ def attn_fwd_fp8(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, q_descale: f
     """e4m3 forward: attention of (q_descale q, k_descale k, v_descale v), D = 128.
     Returns (o bf16, lse fp32) in attn_fwd's layouts."""
     _check_e4m3(q, k, v)
-    B, S, Hq, Hkv, D = _dims(q, k, cu_seqlens)
+    B, S, Hq, Hkv, D = _dims(q, k, cu_seqlens, v)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
+    shape = _lse_shape(B, S, Hq, cu_seqlens is not None)
+    _check_tensor(out, "out", q.shape, torch.bfloat16, q.device)
+    _check_tensor(lse, "lse", shape, torch.float32, q.device)
     if out is None:
         out = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
     if lse is None:
-        shape = (Hq, S) if cu_seqlens is not None else (B, Hq, S)
         lse = torch.empty(shape, dtype=torch.float32, device=q.device)
     st = capi.attn_fwd_fp8(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
                            B, Hq, Hkv, S, D, causal, scale, q_descale, k_descale, v_descale,
@@ -268,8 +321,9 @@ def accumulate_bf16(acc: torch.Tensor, x: torch.Tensor, init: bool = False) -> t
     """acc (fp32) = (0 if init else acc) + x (bf16), element-wise in libattn.so."""
     if not (acc.is_cuda and x.is_cuda and acc.is_contiguous() and x.is_contiguous()):
         raise ValueError("accumulate_bf16 needs contiguous CUDA tensors (there is no CPU path)")
-    if acc.dtype != torch.float32 or x.dtype != torch.bfloat16 or acc.numel() != x.numel():
-        raise ValueError("acc must be fp32 and x bf16 of the same size")
+    if acc.dtype != torch.float32 or x.dtype != torch.bfloat16 or acc.numel() != x.numel() \
+            or acc.device != x.device:
+        raise ValueError("acc must be fp32 and x bf16 of the same size, on one device")
     capi.check(capi.attn_accumulate_bf16(acc.data_ptr(), x.data_ptr(), x.numel(), init,
                                          _stream(x.device)), "attn_accumulate_bf16")
     return acc
@@ -279,6 +333,7 @@ def convert_f32_bf16(x: torch.Tensor, out: Optional[torch.Tensor] = None) -> tor
     """bf16 copy of an fp32 tensor (round to nearest even) in libattn.so."""
     if not (x.is_cuda and x.is_contiguous() and x.dtype == torch.float32):
         raise ValueError("convert_f32_bf16 needs a contiguous fp32 CUDA tensor")
+    _check_tensor(out, "out", x.shape, torch.bfloat16, x.device)
     out = torch.empty(x.shape, dtype=torch.bfloat16, device=x.device) if out is None else out
     capi.check(capi.attn_convert_f32_bf16(out.data_ptr(), x.data_ptr(), x.numel(),
                                           _stream(x.device)), "attn_convert_f32_bf16")

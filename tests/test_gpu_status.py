@@ -87,3 +87,37 @@ def test_calls_leave_the_callers_current_device_alone():
         o1, _ = ops.attn_fwd(q, q, q, causal=True)
     torch.cuda.synchronize(1)
     assert torch.equal(o, o1)
+
+
+@pytest.mark.gpu
+def test_wrapper_rejects_mismatched_tensors_before_launching():
+    """Outputs supplied by the caller, and inputs whose size the kernel takes from q or k,
+    must match exactly: a smaller one would be written or read past its end."""
+    from long_context_attention_fwd_b200 import ops
+    q = torch.randn(1, 256, 4, 64, device="cuda").bfloat16()
+    k = torch.randn(1, 256, 2, 64, device="cuda").bfloat16()
+    o, lse = ops.attn_fwd(q, k, k, causal=True)
+    bad = [
+        lambda: ops.attn_fwd(q, k, k, out=torch.empty(1, 255, 4, 64, device="cuda", dtype=torch.bfloat16)),
+        lambda: ops.attn_fwd(q, k, k, lse=torch.empty(1, 4, 255, device="cuda")),
+        lambda: ops.attn_fwd(q, k, k, lse=torch.empty(1, 4, 256, device="cuda", dtype=torch.float64)),
+        lambda: ops.attn_fwd(q, k, k[:, :, :1].contiguous()),                    # v is not k's shape
+        lambda: ops.attn_bwd(q, k, k, o, lse, q[:, :128].contiguous()),           # dout too short
+        lambda: ops.attn_bwd(q, k, k, o[:, :128].contiguous(), lse, q),           # o too short
+        lambda: ops.attn_bwd(q, k, k, o, lse[:, :2].contiguous(), q),             # lse too small
+        lambda: ops.attn_bwd(q, k, k, o, lse, q, dk=torch.empty_like(q)),         # dk is q's shape
+        lambda: ops.attn_bwd(q, k, k, o, lse, q, workspace=torch.empty(16, device="cpu")),
+        lambda: ops.attn_merge([o, o], [lse, lse], lse=torch.empty(1, 4, 100, device="cuda")),
+        lambda: ops.convert_f32_bf16(torch.zeros(10, device="cuda"),
+                                     out=torch.empty(9, device="cuda", dtype=torch.bfloat16)),
+    ]
+    for i, call in enumerate(bad):
+        with pytest.raises(ValueError):
+            call()
+    # a workspace of another dtype is measured in bytes, not elements
+    need = ops.attn_bwd_workspace_size(q)
+    ws = torch.empty((need + 3) // 4, dtype=torch.float32, device="cuda")
+    dq, dk, dv = ops.attn_bwd(q, k, k, o, lse, q, workspace=ws)
+    dq2, dk2, dv2 = ops.attn_bwd(q, k, k, o, lse, q)
+    torch.cuda.synchronize()
+    assert torch.equal(dk, dk2) and torch.equal(dv, dv2)
