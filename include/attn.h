@@ -27,6 +27,11 @@
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  All work is
  *     asynchronous on that stream; arguments are validated synchronously before
  *     anything is launched, and nothing is launched when validation fails.
+ *   - Work runs on the device that owns the first tensor argument; the entry point
+ *     makes that device current for its launches and, on return, makes the calling
+ *     thread's previous device current again when that device's primary context is
+ *     active (no context is created on a device the process has not used).  The
+ *     stream must belong to the tensors' device.
  *   - No entry point allocates device memory, and no per-call state is kept; the one
  *     exception to "caller-owned memory" is the fixed scratch array attn_bwd_noalloc
  *     works in, which is part of the loaded library.
