@@ -16,6 +16,11 @@ read; attention then runs unchanged on that head group; the second all-to-all tr
 back.  Both Hq and Hkv must be divisible by N (no key/value head replication).  The
 backward sends dO the same way as q and returns dq, dk, dv the same way as o.
 
+Packed batches work the same way: the token stream [T][H][D] of all sequences is cut
+into N equal slices, rank r holding tokens [r*T/N, (r+1)*T/N) whatever sequences they
+belong to.  The exchange gives every rank the whole stream for its heads, so the
+attention runs with the batch's global cu_seqlens, unchanged.
+
 The all-to-alls are torch.distributed collectives (NCCL on GPUs); the layout changes
 around them and the attention itself run in libattn.so.  Nothing reads another GPU's
 memory directly.
@@ -35,23 +40,38 @@ class Hooks:
     """The compute and layout steps; the defaults are this library's kernels.  The CPU
     tests replace them (the fp64 oracle and a plain tensor transpose) to check the
     exchanges on gloo without a GPU."""
-    fwd: Callable = None        # (q, k, v, causal, scale) -> (o, lse)
-    bwd: Callable = None        # (q, k, v, o, lse, do, causal, scale) -> (dq, dk, dv)
+    fwd: Callable = None        # (q, k, v, causal, scale[, cu_seqlens]) -> (o, lse)
+    bwd: Callable = None        # (q, k, v, o, lse, do, causal, scale[, cu_seqlens]) -> grads
     transpose: Callable = None  # (x, n_outer, n_inner) -> x as [n_inner][n_outer][block]
 
     def resolved(self) -> "Hooks":
         return Hooks(
-            fwd=self.fwd or (lambda q, k, v, c, s: ops.attn_fwd(q, k, v, causal=c, scale=s)),
-            bwd=self.bwd or (lambda q, k, v, o, l, do, c, s:
-                             ops.attn_bwd(q, k, v, o, l, do, causal=c, scale=s)),
+            fwd=self.fwd or (lambda q, k, v, c, s, cu=None:
+                             ops.attn_fwd(q, k, v, causal=c, scale=s, cu_seqlens=cu)),
+            bwd=self.bwd or (lambda q, k, v, o, l, do, c, s, cu=None:
+                             ops.attn_bwd(q, k, v, o, l, do, causal=c, scale=s, cu_seqlens=cu)),
             transpose=self.transpose or ops.transpose_blocks)
 
 
 def check_dense(*ts) -> None:
     for t in ts:
         if t.dim() != 4:
-            raise ValueError("the Ulysses wrappers take dense [B][C][H][D] chunks (packed "
-                             "batches are not supported)")
+            raise ValueError("dense Ulysses inputs are [B][C][H][D] chunks")
+
+
+def check_packed(*ts) -> None:
+    for t in ts:
+        if t.dim() != 3:
+            raise ValueError("packed Ulysses inputs are [Tc][H][D] slices of the token stream")
+
+
+def _as_batch(x: torch.Tensor) -> torch.Tensor:
+    """A packed slice [Tc][H][D] seen as a one-sequence dense batch [1][Tc][H][D]."""
+    return x.view(1, *x.shape) if x.dim() == 3 else x
+
+
+def _call(fn, args, cu):
+    return fn(*args) if cu is None else fn(*args, cu)
 
 
 def check_split(Hq: int, Hkv: int, N: int) -> None:
@@ -100,44 +120,55 @@ def _all_to_all(x: torch.Tensor, group) -> torch.Tensor:
 
 class _UlyssesAttention(torch.autograd.Function):
     @staticmethod
-    def forward(ctx, q, k, v, causal, scale, group, hooks):
+    def forward(ctx, q, k, v, causal, scale, group, hooks, cu_seqlens):
         import torch.distributed as dist
         N = dist.get_world_size(group)
-        check_dense(q, k, v)
-        check_split(q.shape[2], k.shape[2], N)
+        packed = cu_seqlens is not None
+        (check_packed if packed else check_dense)(q, k, v)
+        check_split(q.shape[-2], k.shape[-2], N)
         tr = hooks.transpose
 
-        def to_heads(x):
-            return recv_to_full(_all_to_all(seq_to_send(x, N, tr), group), tr)
+        def to_heads(x):   # -> the whole sequence (stream) of this rank's heads
+            f = recv_to_full(_all_to_all(seq_to_send(_as_batch(x), N, tr), group), tr)
+            return f.view(f.shape[1:]) if packed else f
+
+        def to_seq(y, shape):   # -> this rank's chunk (slice), all heads, in `shape`
+            return recv_to_seq(_all_to_all(full_to_send(_as_batch(y), N, tr), group),
+                               tr).view(shape)
 
         qf, kf, vf = to_heads(q), to_heads(k), to_heads(v)
-        o_loc, lse_loc = hooks.fwd(qf, kf, vf, causal, scale)
-        o = recv_to_seq(_all_to_all(full_to_send(o_loc, N, tr), group), tr)
+        o_loc, lse_loc = _call(hooks.fwd, (qf, kf, vf, causal, scale), cu_seqlens)
+        o = to_seq(o_loc, q.shape)
         ctx.save_for_backward(qf, kf, vf, o_loc, lse_loc)
         ctx.causal, ctx.scale, ctx.group, ctx.hooks, ctx.N = causal, scale, group, hooks, N
+        ctx.cu, ctx.to_heads, ctx.to_seq = cu_seqlens, to_heads, to_seq
+        ctx.shapes = (q.shape, k.shape, v.shape)
         return o
 
     @staticmethod
     def backward(ctx, do):
         qf, kf, vf, o_loc, lse_loc = ctx.saved_tensors
-        N, tr, group = ctx.N, ctx.hooks.transpose, ctx.group
-        dof = recv_to_full(_all_to_all(seq_to_send(do.contiguous(), N, tr), group), tr)
-        grads = ctx.hooks.bwd(qf, kf, vf, o_loc, lse_loc, dof, ctx.causal, ctx.scale)
-        dq, dk, dv = (recv_to_seq(_all_to_all(full_to_send(g, N, tr), group), tr)
-                      for g in grads)
-        return dq, dk, dv, None, None, None, None
+        dof = ctx.to_heads(do.contiguous())
+        grads = _call(ctx.hooks.bwd, (qf, kf, vf, o_loc, lse_loc, dof, ctx.causal, ctx.scale),
+                      ctx.cu)
+        dq, dk, dv = (ctx.to_seq(g, t) for g, t in zip(grads, ctx.shapes))
+        return dq, dk, dv, None, None, None, None, None
 
 
 def ulysses_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = True,
                       scale: Optional[float] = None, group=None,
-                      hooks: Optional[Hooks] = None) -> torch.Tensor:
-    """Attention of this rank's sequence chunk (q [B][C][Hq][D], k/v [B][C][Hkv][D], the
-    chunks of all ranks in rank order forming the sequence) over the whole sequence,
-    autograd-aware.  Returns o [B][C][Hq][D]."""
+                      hooks: Optional[Hooks] = None,
+                      cu_seqlens: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Attention of this rank's sequence chunk over the whole sequence, autograd-aware.
+    Dense: q [B][C][Hq][D], k/v [B][C][Hkv][D], the chunks of all ranks in rank order
+    forming the sequence; returns o [B][C][Hq][D].  Packed (cu_seqlens given): q
+    [Tc][Hq][D], k/v [Tc][Hkv][D] are this rank's slice of the token stream and
+    cu_seqlens the whole batch's offsets (the same on every rank); returns o [Tc][Hq][D]."""
     import torch.distributed as dist
     if hooks is None and dist.get_world_size(group) == 1:
-        return ops.attention(q, k, v, causal=causal, scale=scale)
-    return _UlyssesAttention.apply(q, k, v, causal, scale, group, (hooks or Hooks()).resolved())
+        return ops.attention(q, k, v, causal=causal, scale=scale, cu_seqlens=cu_seqlens)
+    return _UlyssesAttention.apply(q, k, v, causal, scale, group, (hooks or Hooks()).resolved(),
+                                   cu_seqlens)
 
 
 def _emulated_all_to_all(sends: List[torch.Tensor]) -> List[torch.Tensor]:
@@ -147,37 +178,46 @@ def _emulated_all_to_all(sends: List[torch.Tensor]) -> List[torch.Tensor]:
 
 def ulysses_attention_single_device(q, k, v, world: int, causal: bool = True,
                                     scale: Optional[float] = None, do=None,
-                                    hooks: Optional[Hooks] = None):
+                                    hooks: Optional[Hooks] = None,
+                                    cu_seqlens: Optional[torch.Tensor] = None):
     """Every rank of a `world`-rank Ulysses group, run one after another on this device
-    from the full tensors (q [B][S][Hq][D], k/v [B][S][Hkv][D]): the same layout steps and
-    per-head-group attention as ulysses_attention, with the all-to-alls done as plain
-    copies.  Returns o, or (o, dq, dk, dv) when `do` is given."""
-    check_dense(q, k, v)
+    from the full tensors (dense q [B][S][Hq][D], k/v [B][S][Hkv][D]; packed q [T][Hq][D],
+    k/v [T][Hkv][D] with cu_seqlens): the same layout steps and per-head-group attention
+    as ulysses_attention, with the all-to-alls done as plain copies.  Returns o, or
+    (o, dq, dk, dv) when `do` is given."""
+    packed = cu_seqlens is not None
+    (check_packed if packed else check_dense)(q, k, v)
     hooks = (hooks or Hooks()).resolved()
     tr = hooks.transpose
-    B, S = q.shape[0], q.shape[1]
-    check_split(q.shape[2], k.shape[2], world)
+    q4, k4, v4 = _as_batch(q), _as_batch(k), _as_batch(v)
+    S = q4.shape[1]
+    check_split(q4.shape[2], k4.shape[2], world)
     if S % world:
-        raise ValueError("sequence length must be divisible by the number of ranks")
+        raise ValueError("sequence length (packed: token count) must be divisible by the "
+                         "number of ranks")
     C = S // world
 
     def chunks(t):
         return [t[:, r * C:(r + 1) * C].contiguous() for r in range(world)]
 
     def to_heads(t):
-        sends = [seq_to_send(x, world, tr) for x in chunks(t)]
-        return [recv_to_full(r, tr) for r in _emulated_all_to_all(sends)]
+        sends = [seq_to_send(x, world, tr) for x in chunks(_as_batch(t))]
+        full = [recv_to_full(r, tr) for r in _emulated_all_to_all(sends)]
+        return [f.view(f.shape[1:]) for f in full] if packed else full
 
-    def to_seq(ys):
-        sends = [full_to_send(y, world, tr) for y in ys]
-        return torch.cat([recv_to_seq(r, tr) for r in _emulated_all_to_all(sends)], dim=1)
+    def to_seq(ys, like):
+        sends = [full_to_send(_as_batch(y), world, tr) for y in ys]
+        out = torch.cat([recv_to_seq(r, tr) for r in _emulated_all_to_all(sends)], dim=1)
+        return out.view(like.shape)
 
     qf, kf, vf = to_heads(q), to_heads(k), to_heads(v)
-    outs = [hooks.fwd(qf[p], kf[p], vf[p], causal, scale) for p in range(world)]
-    o = to_seq([x[0] for x in outs])
+    outs = [_call(hooks.fwd, (qf[p], kf[p], vf[p], causal, scale), cu_seqlens)
+            for p in range(world)]
+    o = to_seq([x[0] for x in outs], q)
     if do is None:
         return o
     dof = to_heads(do)
-    grads = [hooks.bwd(qf[p], kf[p], vf[p], outs[p][0], outs[p][1], dof[p], causal, scale)
+    grads = [_call(hooks.bwd, (qf[p], kf[p], vf[p], outs[p][0], outs[p][1], dof[p], causal,
+                               scale), cu_seqlens)
              for p in range(world)]
-    return (o,) + tuple(to_seq([g[i] for g in grads]) for i in range(3))
+    return (o,) + tuple(to_seq([g[i] for g in grads], t) for i, t in enumerate((q, k, v)))

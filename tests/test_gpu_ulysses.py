@@ -96,3 +96,39 @@ def test_ulysses_full_size_matches_unsplit_kernels(idx, world):
     og = f64(bits_of(o)).reshape(w.S, w.Hq, w.D)[rows[:, 2], rows[:, 1]]
     rep = o_error_report(og, o_r, oa_r)
     assert rep["n_over_model"] == 0 and rep["max_abs"] <= 1e-2, rep
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("lens,world", [([300, 1, 0, 211, 128], 2), (None, 4)],
+                         ids=["packed_small_N2", "packed32K_N4"])
+def test_ulysses_packed_matches_unsplit_kernels(lens, world):
+    """Packed batches: every rank holds a slice of the token stream that cuts sequences
+    mid-way; after the exchange each head group runs the packed kernels with the batch's
+    global cu_seqlens, so o, dk and dv equal the unsplit packed kernels bit for bit."""
+    from long_context_attention_fwd_b200 import ops
+    from long_context_attention_fwd_b200 import ulysses as U
+    w = I.workload(3) if lens is None else make_case(0, 4, 2, 0, 128, True, lens=lens, seed=61)
+    x = I.make_inputs(w)
+    T = w.tokens
+    q, k, v, do = (torch_bf16(x[n]).view(T, h, w.D) for n, h in
+                   (("q", w.Hq), ("k", w.Hkv), ("v", w.Hkv), ("do", w.Hq)))
+    cu = torch.from_numpy(x["cu_seqlens"]).cuda()
+    o, dq, dk, dv = U.ulysses_attention_single_device(q, k, v, world, w.causal, w.softmax_scale,
+                                                      do=do, cu_seqlens=cu)
+    of, lf = ops.attn_fwd(q, k, v, causal=w.causal, scale=w.softmax_scale, cu_seqlens=cu)
+    dqf, dkf, dvf = ops.attn_bwd(q, k, v, of, lf, do, causal=w.causal, scale=w.softmax_scale,
+                                 cu_seqlens=cu)
+    torch.cuda.synchronize()
+    assert _same_bits(o, of)
+    assert _same_bits(dk, dkf) and _same_bits(dv, dvf)
+    a, b = dq.float(), dqf.float()
+    assert float((a - b).norm() / b.norm()) <= 2.0 ** -8
+    if lens is not None:   # small: the whole result against the oracle
+        qn, kn, vn, don, kw = oracle_args(w, x)
+        o_r, _ = oracle.fwd(qn, kn, vn, True, w.softmax_scale, **kw)
+        oa_r, _ = oracle.fwd(qn, kn, np.abs(vn), True, w.softmax_scale, **kw)
+        rep = o_error_report(f64(bits_of(o)).reshape(T, w.Hq, w.D), o_r, oa_r)
+        assert rep["n_over_model"] == 0 and rep["max_abs"] <= 1e-2, rep
+        g_r = oracle.bwd(qn, kn, vn, don, True, w.softmax_scale, **kw)
+        for got, ref, H in ((dq, g_r[0], w.Hq), (dk, g_r[1], w.Hkv), (dv, g_r[2], w.Hkv)):
+            assert rel_l2(f64(bits_of(got)).reshape(T, H, w.D), ref) <= TOL_GRAD
