@@ -159,25 +159,28 @@ def summarize_clocks(lines, t0: float, t1: float) -> dict:
 
 
 class ClockSampler:
-    """nvidia-smi every 50 ms into clocks_bench_<pid>.csv, summarised over the timed
-    region's wall-clock window.  The log goes to $ATTN_BENCH_CLOCKS_DIR when set, else to
-    the system's temporary directory."""
+    """nvidia-smi every 50 ms, read through a pipe (no file) by a thread that keeps the
+    pipe drained, and summarised over the timed region's wall-clock window."""
 
     def __init__(self, index: int):
-        import tempfile
         self.index = index
         self.proc = None
-        folder = os.environ.get("ATTN_BENCH_CLOCKS_DIR") or tempfile.gettempdir()
-        self.path = os.path.join(folder, f"clocks_bench_{os.getpid()}.csv")
+        self.lines = []
+        self.reader = None
+
+    def _drain(self):
+        for line in self.proc.stdout:
+            self.lines.append(line)
 
     def start(self):
+        import threading
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
-            self.f = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={CLOCK_FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "50"], stdout=self.f,
-                stderr=subprocess.DEVNULL)
+                 "--format=csv,noheader,nounits", "-lms", "50"], stdout=subprocess.PIPE,
+                stderr=subprocess.DEVNULL, text=True)
+            self.reader = threading.Thread(target=self._drain, daemon=True)
+            self.reader.start()
         except Exception:
             self.proc = None
 
@@ -190,9 +193,8 @@ class ClockSampler:
             self.proc.wait(timeout=5)
         except Exception:
             self.proc.kill()
-        self.f.close()
-        with open(self.path) as f:
-            return summarize_clocks(f.readlines(), t0, t1)
+        self.reader.join(timeout=5)
+        return summarize_clocks(list(self.lines), t0, t1)
 
 
 # ---------------------------------------------------------------- CPU oracle
