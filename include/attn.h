@@ -41,6 +41,9 @@
  *   - Device-side waits are bounded; a wait that times out makes the kernel skip
  *     its remaining work and records the event in a sticky status word that
  *     attn_device_status reports.
+ *   - The library looks up the device addresses of its own device-side variables (the
+ *     status word, attn_bwd_noalloc's scratch array) once per device and keeps them;
+ *     a cudaDeviceReset between calls is not supported.
  */
 #ifndef ATTN_H_
 #define ATTN_H_

@@ -21,6 +21,7 @@ ATTN_ERR_UNSUPPORTED = 2
 ATTN_ERR_MISALIGNED = 3
 ATTN_ERR_CUDA = 4
 ATTN_ERR_TIMEOUT = 5
+ATTN_BWD_NOALLOC_MAX_BYTES = 64 << 20  # the header's define of the same name
 
 
 class AttnError(RuntimeError):

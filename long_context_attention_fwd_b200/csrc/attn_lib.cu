@@ -837,14 +837,21 @@ extern "C" attn_status attn_bwd_noalloc(const void* q, const void* k, const void
                                         const int32_t* cu_seqlens, void* stream) {
   DeviceRestore restore_device;
   const size_t need = attn_bwd_workspace_size(B, Hq, S, D, cu_seqlens);
-  if (need == 0) return ATTN_ERR_INVALID_ARG;  // the same size checks attn_bwd applies
+  if (need == 0) {  // the same size checks attn_bwd applies
+    snprintf(g_last_error, sizeof(g_last_error),
+             "attn_bwd_noalloc: invalid sizes (B=%d Hq=%d S=%d D=%d)", B, Hq, S, D);
+    return ATTN_ERR_INVALID_ARG;
+  }
   if (need > size_t(ATTN_BWD_NOALLOC_MAX_BYTES)) {
     snprintf(g_last_error, sizeof(g_last_error),
              "attn_bwd_noalloc: workspace of %zu bytes exceeds the static scratch of %zu bytes",
              need, size_t(ATTN_BWD_NOALLOC_MAX_BYTES));
     return ATTN_ERR_INVALID_ARG;
   }
-  if (!q) return ATTN_ERR_INVALID_ARG;
+  if (!q) {
+    snprintf(g_last_error, sizeof(g_last_error), "attn_bwd_noalloc: q is a null pointer");
+    return ATTN_ERR_INVALID_ARG;
+  }
   // Set-up, once per device and with that device current: the array's name is only a
   // host-side stand-in, so its device address is looked up and cached.
   cudaPointerAttributes attr;

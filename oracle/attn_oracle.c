@@ -15,7 +15,7 @@
  * exactly this result ("numerically consistent"), so this plain definition is the
  * thing the GPU path must reproduce up to rounding.
  *
- * Readings where the page is silent (each listed in the design notes):
+ * Readings where the page is silent (the plainest one that fits the rest of the page):
  *   - scores carry a factor `scale` (1/sqrt(D) by default): s_ij = scale * q_i . k_j;
  *   - causal: key j is visible to query i iff j <= i, positions counted from the start
  *     of the query's own sequence; packed sequences never see each other;

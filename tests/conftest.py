@@ -39,3 +39,18 @@ def _short_device_waits():
     except Exception:
         pass
     yield
+
+
+def pytest_terminal_summary(terminalreporter):
+    """Prints the parity figures the GPU tests recorded (strict O counts, gradient
+    errors), so that a run's output shows them whether the tests passed or not."""
+    try:
+        from helpers import PARITY_LOG
+    except Exception:
+        return
+    if not PARITY_LOG:
+        return
+    import json
+    terminalreporter.section("parity figures")
+    for label, metrics in PARITY_LOG:
+        terminalreporter.write_line(f"{label}: {json.dumps(metrics, sort_keys=True)}")
