@@ -729,8 +729,48 @@ def run_gpu(args, w: I.Workload):
     return 0
 
 
+def run_profile_case(args):
+    """One launch of the forward and/or backward on a reduced synthetic problem, for ncu
+    captures that must stay small (a few GB on the device, one launch of each kernel):
+    --profile B,Hq,Hkv,S,D [--profile-op fwd|bwd|both] [--profile-outliers].  Inputs are
+    drawn on the GPU (N(0,1) * 0.5, or N(0,1) with 1% of q, k entries x8); the backward
+    needs the forward's output, so --profile-op bwd also launches the forward once."""
+    import torch
+    from long_context_attention_fwd_b200 import capi, ops
+    B, Hq, Hkv, S, D = (int(x) for x in args.profile.split(","))
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev).manual_seed(20261203)
+    mult = 1.0 if args.profile_outliers else 0.5
+
+    def draw(H, outliers):
+        x = torch.randn((B, S, H, D), generator=g, device=dev) * mult
+        if outliers:
+            x = torch.where(torch.rand(x.shape, generator=g, device=dev) < 0.01, x * 8, x)
+        return x.bfloat16()
+
+    q, k = draw(Hq, args.profile_outliers), draw(Hkv, args.profile_outliers)
+    v, do = draw(Hkv, False), draw(Hq, False)
+    scale = D ** -0.5
+    o, lse = ops.attn_fwd(q, k, v, causal=True, scale=scale)
+    if args.profile_op in ("fwd", "both"):
+        ops.attn_fwd(q, k, v, causal=True, scale=scale, out=o, lse=lse)
+    if args.profile_op in ("bwd", "both"):
+        ops.attn_bwd(q, k, v, o, lse, do, causal=True, scale=scale)
+    torch.cuda.synchronize()
+    st, site = capi.attn_device_status(None)
+    if st != capi.ATTN_OK:
+        raise RuntimeError(f"device status {capi.strerror(st)} site={site:#x}")
+    print(json.dumps({"profile_case": [B, Hq, Hkv, S, D], "op": args.profile_op,
+                      "outliers": bool(args.profile_outliers), "status": "ok"}))
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
+    ap.add_argument("--profile", default=None, metavar="B,Hq,Hkv,S,D",
+                    help="one launch on a reduced synthetic problem, for ncu captures")
+    ap.add_argument("--profile-op", default="both", choices=["fwd", "bwd", "both"])
+    ap.add_argument("--profile-outliers", action="store_true")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
@@ -746,6 +786,8 @@ def main():
     ap.add_argument("--no-ring", action="store_true",
                     help="skip the Ring-attention measurements (merge kernel, 1-GPU ring forward)")
     args = ap.parse_args()
+    if args.profile:
+        return run_profile_case(args)
     w = I.workload(args.workload)
     if args.impl == "reference":
         return run_reference(args, w)

@@ -136,8 +136,8 @@ attn_status attn_bwd_noalloc(const void* q, const void* k, const void* v, const 
                              const int32_t* cu_seqlens, void* stream);
 
 /* Bytes of device workspace attn_decode needs (0 for invalid sizes).  It holds the
- * per-split partial results: 2 * nsplit partials of B*Hq rows (bf16 o and fp32 lse), where
- * nsplit is fixed by (B, Hkv, Lmax). */
+ * per-split partial results, 2 * nsplit partials of B*Hq rows (bf16 o and fp32 lse) where
+ * nsplit is fixed by (B, Hkv, Lmax), and one 8-byte arrival word per (sequence, kv head). */
 size_t attn_decode_workspace_size(int B, int Hq, int Hkv, int Lmax, int D);
 
 /* Decode attention over a key/value cache: one new query token per sequence attends to
@@ -152,8 +152,13 @@ size_t attn_decode_workspace_size(int B, int Hq, int Hkv, int Lmax, int D);
  *     cache_len[b] are never used, whatever they hold.  cache_len[b] = 0 gives o = 0 and
  *     lse = -inf.
  *   - The cache is split along the keys; every split writes a partial (o, lse) into
- *     `workspace` (>= attn_decode_workspace_size bytes, 256-byte aligned, caller-owned,
- *     no initialisation needed) and attn_merge's kernel combines them exactly.
+ *     `workspace` (>= attn_decode_workspace_size bytes, 256-byte aligned, caller-owned),
+ *     and the last split of each (sequence, kv head) to finish combines them exactly, in
+ *     the same launch.  The splits count their arrivals in the workspace's arrival
+ *     words; each word carries a 48-bit tag of the call, so the workspace needs no
+ *     initialisation (leftover contents are taken for another call's, except with
+ *     probability 2^-48 per word), and a call leaves its words cleared.  Two calls
+ *     whose work overlaps on the GPU must not share a workspace.
  *   - D in {64, 128}; Hq a multiple of Hkv with Hq/Hkv <= 128; B*Lmax and B*Hq < 2^31.
  *   - Pointers as in every entry point (16-byte aligned tensors, 4-byte lse/cache_len).
  *   - Deterministic. */
@@ -253,6 +258,12 @@ attn_status attn_selftest_wait_timeout(unsigned long long timeout_ns, void* stre
  * c is fp32. */
 attn_status attn_selftest_umma(int mode, int D, const void* a, const void* b, const float* p,
                                const void* at, float* c, void* stream);
+
+/* Self-test of the exponential the forward kernel computes on the FMA pipe for a share
+ * of its probabilities (no page counterpart): y[i] = 2^x[i] by that polynomial route,
+ * for n values (x, y DEVICE fp32, 16-byte aligned, n > 0 and even).  Maximum relative
+ * error 2^-18 for x in [-125, 64]; below -125 the result is about 2^-125. */
+attn_status attn_selftest_exp2(const float* x, float* y, long long n, void* stream);
 
 /* Description of the last failing CUDA call this library made on the calling thread
  * ("" if none): the call's name and the CUDA error string.  Static per-thread

@@ -68,6 +68,7 @@ _SIGNATURES = {
     "attn_transpose_blocks": (_i, [_vp, _vp, ctypes.c_longlong, ctypes.c_longlong,
                                    ctypes.c_longlong, _vp]),
     "attn_merge": (_i, [_vp, _vp, _i, _vp, _fp, _i, _i, _i, _i, _vp]),
+    "attn_selftest_exp2": (_i, [_fp, _fp, ctypes.c_longlong, _vp]),
     "attn_bwd_noalloc": (_i, [_vp, _vp, _vp, _vp, _fp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
                               ctypes.c_float, _vp, _vp]),
 }
@@ -205,6 +206,10 @@ def attn_selftest_umma(mode, D, a, b, p, at, c, stream=None) -> int:
 
 def attn_selftest_umma_fp8(mode, a, b, pin, pq, c, stream=None) -> int:
     return lib().attn_selftest_umma_fp8(mode, a, b, pin, pq, c, stream)
+
+
+def attn_selftest_exp2(x, y, n, stream=None) -> int:
+    return lib().attn_selftest_exp2(x, y, int(n), stream)
 
 
 def attn_version() -> int:

@@ -84,7 +84,12 @@ struct Cfg {
   static constexpr int SLACK = (SMEM_BYTES + 1024 <= kMaxDyn) ? 1024 : (kMaxDyn - SMEM_BYTES);
   static constexpr int SMEM_ALLOC = SMEM_BYTES + SLACK;
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DQ = 128, COL_DV = 256, COL_DK = 256 + D;
+  // D = 128 fills TMEM with S^T, dP^T, dV, dK, so the dQ tile shares dP^T's columns and
+  // the next dP^T waits for the dQ drain.  D = 64 leaves room for dQ columns of its own.
+  static constexpr bool DQ_ALIAS = D == 128;
+  static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DV = 256, COL_DK = 256 + D;
+  static constexpr uint32_t COL_DQ = DQ_ALIAS ? COL_DP : 256 + 2 * D;
+  static_assert(COL_DQ + D <= TMEM_COLS && (DQ_ALIAS || COL_DQ >= COL_DK + D), "TMEM budget");
   static_assert(SMEM_BYTES <= kMaxDyn, "shared memory budget");
 };
 
@@ -339,22 +344,24 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       // P^T and dS^T halves sit in TMEM columns [0, 32) and [96, 128) of their regions
       // (warps 0-3 / warps 4-7, bf16 pairs): A-operand column of 16-row step kk.
       auto a_col = [](int kk) -> uint32_t { return kk < 4 ? kk * 8 : 96 + (kk - 4) * 8; };
+      // Per query tile: dP^T first (it needs neither P nor dS, so the dS step can start as
+      // soon as P is done), then dV, the next S^T, dK and dQ.
       for (int it = 0; it < iters && ok; ++it) {
         const int st = it & 1;
         const uint32_t ph = (it >> 1) & 1;
         const uint32_t qb = smem_u32(smem + C::OFF_Q + st * C::TILE);
         const uint32_t dob = smem_u32(smem + C::OFF_DO + st * C::TILE);
         if (!(ok = mbar_wait(&do_full[st], ph, wc, kSiteDoFull))) break;
+        if (C::DQ_ALIAS && it > 0 && !(ok = mbar_wait(dq_free, (it - 1) & 1, wc, kSiteDqFree))) break;
+        tc_fence_after();
+        issue_T(C::COL_DP, vb, dob);  // dP^T = V dO^T (over dS^T of the previous tile, or dQ)
+        mma_commit(dp_full);
         if (!(ok = mbar_wait(p_full, it & 1, wc, kSitePFull))) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)  // dV += P^T dO
           mma_ts(tmem + C::COL_DV, tmem + C::COL_S + a_col(kk), sdesc_sw128(dob + kk * 2048, kSlab, 1024),
                  idKV, (it > 0 || kk > 0) ? 1u : 0u);
-        if (it > 0 && !(ok = mbar_wait(dq_free, (it - 1) & 1, wc, kSiteDqFree))) break;
-        tc_fence_after();
-        issue_T(C::COL_DP, vb, dob);  // dP^T = V dO^T (into the columns dQ was drained from)
-        mma_commit(dp_full);
         mma_commit(&do_empty[st]);
         if (it + 1 < iters) {
           if (!(ok = mbar_wait(&q_full[st ^ 1], ((it + 1) >> 1) & 1, wc, kSiteQFull))) break;
@@ -369,6 +376,8 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           mma_ts(tmem + C::COL_DK, tmem + C::COL_DP + a_col(kk), sdesc_sw128(qb + kk * 2048, kSlab, 1024),
                  idKV, (it > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&q_empty[st]);
+        if (!C::DQ_ALIAS && it > 0 && !(ok = mbar_wait(dq_free, (it - 1) & 1, wc, kSiteDqFree))) break;
+        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)  // dQ_tile = dS K
           mma_ss(tmem + C::COL_DQ, sdesc_sw128(dsb + kk * 2048, 16384, 1024),

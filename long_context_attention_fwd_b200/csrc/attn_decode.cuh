@@ -25,8 +25,16 @@
 // Cache rows past a sequence's length are never used: their scores are masked to -inf, and
 // the rows of the last V tile past the length are zeroed in shared memory before its PV
 // product (whatever the cache holds there, 0 * NaN would otherwise poison O).
+//
+// The last CTA of a (sequence, kv head) to finish combines the partials of every split
+// into o and lse (the exact log-sum-exp rule of attn_merge), so a decode step is one
+// launch.  CTAs count their arrivals on a per-(sequence, kv head) word in the caller's
+// workspace, which may hold anything when the call starts: the word carries a 48-bit tag
+// of the call that wrote it, and a word with another tag counts as zero.  The merging CTA
+// clears its word again, so the next call (or a replay of the same launch) starts clean.
 #pragma once
 #include <cuda_bf16.h>
+#include "attn_merge.cuh"
 #include "sm100_ptx.cuh"
 
 namespace attn_sm100 {
@@ -43,6 +51,7 @@ constexpr int kRegsCompute = 216;
 static_assert(128 * kRegsControl + 256 * kRegsCompute <= kThreads * kRegsLaunch, "register split");
 constexpr float kRescaleThreshold = 8.0f;
 constexpr int kSlab = 128 * 128;
+constexpr int kMaxParts = 256;  // partials per row: 2 streams x at most 128 splits
 
 struct Params {
   const int32_t* cache_len;  // [B] (device); clamped to [0, Lmax]
@@ -51,6 +60,10 @@ struct Params {
   int Hq, G, Hkv, Lmax;
   int nsplit, tps;           // splits per (sequence, kv head); tiles per split
   int rows;                  // B * Hq (row stride between partials)
+  unsigned long long* ctr;   // [B * Hkv] arrival words (caller workspace, any initial value)
+  unsigned long long tag;    // this call's tag: nonzero, below 2^48
+  __nv_bfloat16* o;          // [B * Hq][D] result
+  float* lse;                // [B * Hq]
   float scale_log2;
   unsigned* status;
   unsigned long long timeout_ns;
@@ -77,8 +90,96 @@ struct Cfg {
 
 enum : unsigned {
   kSiteKEmpty = 0x300, kSiteVEmpty, kSiteQFull, kSiteKFull, kSiteVFull, kSitePFull, kSiteSFull,
-  kSiteOFinal, kSiteVRaw, kSiteDrainQ, kSiteDrainK, kSiteDrainV, kSiteDrainVRaw, kSiteDrainMMA
+  kSiteOFinal, kSiteVRaw, kSiteDrainQ, kSiteDrainK, kSiteDrainV, kSiteDrainVRaw, kSiteDrainMMA,
+  kSiteTicket
 };
+
+// Counts this CTA's arrival on `word`: bits 63..16 hold the tag of the call that last
+// counted there, bits 15..0 its count.  A word with another tag (an earlier call, or
+// memory never written, which matches a given 48-bit tag with probability 2^-48) counts
+// as zero.  Returns the count including this arrival, or -1 if the compare-and-swap
+// loop gave up (it retries only while other CTAs of the same call arrive at once).
+__device__ __forceinline__ int arrive_count(unsigned long long* word, unsigned long long tag) {
+  unsigned long long cur = atomicAdd(word, 0ull);
+#pragma unroll 1
+  for (int i = 0; i < (1 << 16); ++i) {
+    const unsigned long long want = (cur >> 16) == tag ? cur + 1 : ((tag << 16) | 1ull);
+    const unsigned long long prev = atomicCAS(word, cur, want);
+    if (prev == cur) return int(want & 0xFFFFull);
+    cur = prev;
+  }
+  return -1;
+}
+
+// Combines the nparts partials of rows row0 .. row0 + G - 1 into p.o and p.lse, with all
+// kThreads threads of the CTA: LSE = ln sum_j exp(LSE_j), O = sum_j exp(LSE_j - LSE) O_j
+// (weights and sums in fp32, one bf16 rounding).  Partials are read through L2 (another
+// CTA wrote most of them).  `scratch` is shared memory the kernel no longer uses.
+template <int D>
+__device__ void merge_rows(const Params& p, int row0, int G, int nparts, uint8_t* scratch) {
+  constexpr int TPR = D / 8;               // threads per row: one 16-byte column group each
+  constexpr int NGRP = kThreads / TPR;     // thread groups
+  float* s_m = reinterpret_cast<float*>(scratch);   // [128] row maximum of the partial LSEs
+  float* s_inv = s_m + 128;                          // [128] 1 / sum of the weights
+  float* s_acc = s_inv + 128;                        // [NGRP][TPR][8] partial sums
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // Per row (one warp each): the largest partial LSE, and the weight sum relative to it.
+  for (int r = warp; r < G; r += kThreads / 32) {
+    const int row = row0 + r;
+    float m = -INFINITY;
+    for (int j = lane; j < nparts; j += 32) m = fmaxf(m, __ldcg(p.lse_part + size_t(j) * p.rows + row));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    float l = 0.f;
+    if (m != -INFINITY)
+      for (int j = lane; j < nparts; j += 32) l += expf(__ldcg(p.lse_part + size_t(j) * p.rows + row) - m);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+    if (lane == 0) {
+      s_m[r] = m;
+      s_inv[r] = (m == -INFINITY) ? 0.f : 1.f / l;
+      p.lse[row] = (m == -INFINITY) ? -INFINITY : m + logf(l);
+    }
+  }
+  __syncthreads();
+  // Rows in passes of rp; the partials of a row are spread over nsub thread groups.
+  const int rp = G < NGRP ? G : NGRP;
+  const int nsub = NGRP / rp;
+  const int grp = threadIdx.x / TPR, c = threadIdx.x % TPR;
+  const size_t pstride = size_t(p.rows) * TPR;  // uint4 stride between partials
+  for (int r0 = 0; r0 < G; r0 += rp) {
+    const int r = r0 + grp % rp, sub = grp / rp;
+    if (sub < nsub && r < G) {
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      const float m = s_m[r];
+      if (m != -INFINITY) {
+        const uint4* ob = reinterpret_cast<const uint4*>(p.o_part) + size_t(row0 + r) * TPR + c;
+        const float* lb = p.lse_part + row0 + r;
+#pragma unroll 4
+        for (int j = sub; j < nparts; j += nsub)
+          merge::acc_bf16x8(acc, __ldcg(ob + size_t(j) * pstride), expf(__ldcg(lb + size_t(j) * p.rows) - m));
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) s_acc[(grp * TPR + c) * 8 + e] = acc[e];
+    }
+    __syncthreads();
+    if (grp < rp && r0 + grp < G) {
+      const int rr = r0 + grp;
+      float o[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      for (int k = 0; k < nsub; ++k)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) o[e] += s_acc[((grp + k * rp) * TPR + c) * 8 + e];
+      const float inv = s_inv[rr];
+      uint4 y;
+      y.x = pack_bf16x2(o[0] * inv, o[1] * inv);
+      y.y = pack_bf16x2(o[2] * inv, o[3] * inv);
+      y.z = pack_bf16x2(o[4] * inv, o[5] * inv);
+      y.w = pack_bf16x2(o[6] * inv, o[7] * inv);
+      reinterpret_cast<uint4*>(p.o + size_t(row0 + rr) * D)[c] = y;
+    }
+    __syncthreads();
+  }
+}
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -283,6 +384,9 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       mbar_drain_checked(drain, 0, wc, kSiteDrainMMA);
     }
    }
+   // Back to the launch budget for the merge below, which every warp runs (this waits
+   // for the softmax warpgroups' matching decrease).
+   reg_alloc<kRegsLaunch>();
   } else {
     reg_alloc<kRegsCompute>();
     // ------------------------------------------------------------ softmax + partial output
@@ -424,14 +528,33 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         }
       }
     }
+    reg_dealloc<kRegsLaunch>();
   }
 
   // ---- teardown: every role has drained; release tensor memory.
+  __threadfence();  // this CTA's partials are visible device-wide before its arrival counts
   tc_fence_before();
   __syncthreads();
   if (warp == kWarpMMA) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+
+  // ---- the last CTA of this (sequence, kv head) to arrive merges every split's partials.
+  volatile int* s_last = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);
+  if (threadIdx.x == 0) {
+    const int cnt = arrive_count(p.ctr + bg, p.tag);
+    if (cnt < 0) {
+      atomicOr(p.status, kStatusTimeout);
+      atomicCAS(p.status + 1, 0u, kSiteTicket);
+    }
+    *s_last = cnt == p.nsplit;
+    if (cnt == p.nsplit) atomicExch(p.ctr + bg, 0ull);  // clear for the next call
+  }
+  __syncthreads();
+  if (*s_last) {
+    __threadfence();
+    merge_rows<D>(p, row0, p.G, 2 * p.nsplit, smem + C::OFF_K);  // K/V stages are free now
   }
 }
 

@@ -11,7 +11,8 @@
 // Blackwell mapping (one CTA = 256 query rows of one head, as two 128-row tiles):
 //   warp 8      TMA producer: Q tiles once, then K_j / V_j into a ring of NS stages.
 //   warp 9      MMA issuer (one thread): S_t = Q_t K_j^T (SS, fp32 in TMEM) and
-//               O_t += P_t V_j (P read from TMEM as bf16, V from shared memory).
+//               O_t += P_t V_j (P read from TMEM as bf16, V from shared memory; at D = 64
+//               also the row sums of P against the ones columns).
 //   warps 10-11 idle (they complete the control warpgroup for the register split).
 //   warps 0-3   softmax for tile 0, warps 4-7 for tile 1: one thread per query row,
 //               reads S from TMEM, exp2-based online max/sum, writes P (bf16) back
@@ -20,6 +21,14 @@
 // The two tiles ping-pong: while softmax works on one tile the tensor core runs the
 // other tile's PV and the next S, so MMA and exponentials overlap.
 //
+// The exponentials and the MMAs of a tile take about equally long at D = 128, and the
+// exponentials twice as long at D = 64, so the MUFU unit paces the loop.  Two changes
+// take work off it and off the softmax threads:
+//   - a share of the exponentials (Cfg::EMU pairs of every 16) is evaluated by a
+//     polynomial on the FMA pipe (exp2_poly_x2) in tiles without masked scores;
+//   - at D = 64 the normaliser over the bf16 weights comes out of the PV MMA itself, as
+//     16 extra accumulator columns against a column of ones in shared memory.
+//
 // FP8 = true is the e4m3 variant (D = 128): Q, K, V are e4m3 with per-tensor descale
 // factors folded into the softmax scale (q, k) and the epilogue (v); the MMAs are
 // kind::f8f6f4 (K = 32 per instruction, twice the bf16 rate); P is quantised as
@@ -27,6 +36,7 @@
 // -- and O is divided by the sum of exactly those quantised weights, so the factor cancels.
 #pragma once
 #include <cuda_bf16.h>
+#include <type_traits>
 #include "attn_common.cuh"
 #include "sm100_ptx.cuh"
 
@@ -46,6 +56,16 @@ constexpr int kRegsCompute = 216;
 static_assert(128 * kRegsControl + 256 * kRegsCompute <= kThreads * kRegsLaunch, "register split");
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when max grows > 2^8
 constexpr int kSlab = 128 * 128;       // one 128-row x 64-column bf16 swizzled slab (16 KB)
+// Share of the exponentials (pairs out of 16) computed on the FMA pipe, per head dim.
+#ifndef ATTN_FWD_EMU64
+#define ATTN_FWD_EMU64 0
+#endif
+#ifndef ATTN_FWD_EMU128
+#define ATTN_FWD_EMU128 2
+#endif
+#ifndef ATTN_FWD_EMU_FP8
+#define ATTN_FWD_EMU_FP8 0
+#endif
 
 struct Params {
   SeqView sv;
@@ -67,6 +87,15 @@ constexpr float kRescaleThresholdFp8 = 0.5f;
 
 template <int D, bool FP8 = false>
 struct Cfg {
+  // D = 64 (bf16): TMEM has room for 16 more accumulator columns per tile, so the PV MMA
+  // also sums the bf16 weights of every row against a column of ones (N = D + 16): the
+  // normaliser then comes from the tensor core, accumulated and rescaled exactly like O,
+  // instead of a second running sum in the softmax threads.
+  static constexpr bool ONES = !FP8 && D == 64;
+  static constexpr int NPV = ONES ? D + 16 : D;          // N of the PV MMA
+  // Of every 16 probability pairs, EMU are exponentiated on the FMA pipe (exp2_poly_x2)
+  // instead of the MUFU unit, in tiles without masked scores.
+  static constexpr int EMU = FP8 ? ATTN_FWD_EMU_FP8 : (D == 64 ? ATTN_FWD_EMU64 : ATTN_FWD_EMU128);
   static constexpr int ES = FP8 ? 1 : 2;                 // bytes per element
   static constexpr int NS = FP8 ? 4 : ((D == 128) ? 2 : 4);
   static constexpr int SLABS = D * ES / 128;             // 128-byte swizzle rows per tile row
@@ -77,15 +106,24 @@ struct Cfg {
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + 2 * QT_BYTES;
   static constexpr int OFF_V = OFF_K + NS * KV_BYTES;
-  static constexpr int OFF_BAR = OFF_V + NS * KV_BYTES;
+  static constexpr int OFF_ONES = OFF_V + NS * KV_BYTES;  // 128 x 64 bf16 slab (ONES only)
+  static constexpr int OFF_BAR = OFF_ONES + (ONES ? kSlab : 0);
   // q_full, k_full[NS], k_empty[NS], v_full[NS], v_empty[NS], s_full[2], p_full[2], o_final[2], drain
   static constexpr int NBAR = 1 + 4 * NS + 7;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16;
   static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;  // slack for 1024-byte alignment
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O0 = 256, COL_O1 = 256 + D;
+  static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O0 = 256, COL_O1 = ONES ? 384 : 256 + D;
+  static_assert(COL_O1 + NPV <= TMEM_COLS, "TMEM budget");
 };
+
+// Pair i (0..15) of a 32-score chunk is exponentiated on the FMA pipe when this holds:
+// EMU of every 16 pairs, spread evenly.
+template <int EMU>
+__device__ __forceinline__ constexpr bool emu_pair(int i) {
+  return EMU > 0 && ((i + 1) * EMU) / 16 != (i * EMU) / 16;
+}
 
 // Wait-site codes reported in the status word when a wait times out.
 enum : unsigned {
@@ -161,6 +199,18 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
   }
+  if constexpr (C::ONES) {
+    // The ones operand of the row-sum columns: 128 key rows of 64 bf16 (one 128-byte
+    // swizzle row each), element 0 = 1 and the rest 0.  With the 128-byte swizzle the
+    // 16-byte chunk c of row r sits at chunk position c ^ (r % 8), so element 0 of row r
+    // lies at byte 16 * (r % 8) of the row.
+    uint4* ones = reinterpret_cast<uint4*>(smem + C::OFF_ONES);
+    for (int i = threadIdx.x; i < kSlab / 16; i += kThreads) {
+      const int r = i >> 3, c = i & 7;
+      ones[i] = make_uint4(c == (r & 7) ? 0x3F80u : 0u, 0u, 0u, 0u);
+    }
+    fence_async_smem();  // generic-proxy writes, read by the tensor core
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -210,7 +260,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idS = FP8 ? idesc_e4m3_f32(128, 128, 0, 0) : idesc_bf16_f32(128, 128, 0, 0);
-      constexpr uint32_t idPV = FP8 ? idesc_e4m3_f32(128, D, 0, 1) : idesc_bf16_f32(128, D, 0, 1);
+      constexpr uint32_t idPV = FP8 ? idesc_e4m3_f32(128, D, 0, 1) : idesc_bf16_f32(128, C::NPV, 0, 1);
       const uint32_t qb[2] = {smem_u32(smem + C::OFF_Q), smem_u32(smem + C::OFF_Q + C::QT_BYTES)};
       const uint32_t colS[2] = {C::COL_S0, C::COL_S1};
       const uint32_t colO[2] = {C::COL_O0, C::COL_O1};
@@ -229,10 +279,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       };
       auto issue_PV = [&](int t, int st, bool acc) {
         const uint32_t vb = smem_u32(smem + C::OFF_V + st * C::KV_BYTES);
+        // MN-major V: 64-element N blocks kSlab apart; with the ones columns the second
+        // N block is the ones slab, which lies after every V stage.
+        constexpr uint32_t kLbo0 = C::ONES ? uint32_t(C::OFF_ONES - C::OFF_V) : uint32_t(kSlab);
+        const uint32_t lbo = C::ONES ? kLbo0 - uint32_t(st * C::KV_BYTES) : kLbo0;
 #pragma unroll
         for (int kk = 0; kk < C::PSTEPS; ++kk) {
           // K step: 32 bytes of keys = 32 / ES key rows of 128 bytes in the MN-major V tile
-          const uint64_t bdesc = sdesc_sw128(vb + kk * (4096 / C::ES), kSlab, 1024);
+          const uint64_t bdesc = sdesc_sw128(vb + kk * (4096 / C::ES), lbo, 1024);
           if constexpr (FP8)
             mma_ts_f8(tmem + colO[t], tmem + colS[t] + kk * 8, bdesc, idPV, (acc || kk > 0) ? 1u : 0u);
           else
@@ -355,7 +409,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       if (j > 0 && __any_sync(0xffffffffu, need)) {
         uint32_t u[32];
 #pragma unroll 1
-        for (int ch = 0; ch < D / 32; ++ch) {
+        for (int ch = 0; ch < (C::NPV + 31) / 32; ++ch) {  // O, and the row-sum columns
           tmem_ld32(tO + ch * 32, u);
           tmem_wait_ld();
 #pragma unroll
@@ -370,48 +424,75 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const uint64_t cc = f2_pack(c, c), mm = f2_pack(mneg, mneg);
       // Two running sums: of the fp32 probabilities (for the log-sum-exp) and of
       // their bf16 roundings (the values the PV MMA consumes), so that O is
-      // normalised by exactly the weights it was accumulated with.
+      // normalised by exactly the weights it was accumulated with.  With the ones
+      // columns the second sum comes out of the PV MMA instead.
       uint64_t sf[4] = {0, 0, 0, 0}, sb[4] = {0, 0, 0, 0};
       if constexpr (!FP8) {
+        // Tiles with no masked score hand a share of the exponentials to the FMA pipe.
+        auto exps = [&](auto emu_tag) {
+          constexpr bool kEmu = decltype(emu_tag)::value;
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        uint32_t pk[16];
+          for (int ch = 0; ch < 4; ++ch) {
+            uint32_t pk[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          float x0, x1;
-          f2_unpack(f2_fma(f2_pack(s[ch * 32 + 2 * i], s[ch * 32 + 2 * i + 1]), cc, mm), x0, x1);
-          const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-          const uint32_t b = pack_bf16x2(p0, p1);
-          pk[i] = b;
-          sf[i & 3] = f2_add(sf[i & 3], f2_pack(p0, p1));
-          sb[i & 3] = f2_add(sb[i & 3], f2_pack(__uint_as_float(b << 16), __uint_as_float(b & 0xFFFF0000u)));
-        }
-        tmem_st16(tS + ch * 16, pk);
-      }
+            for (int i = 0; i < 16; ++i) {
+              const uint64_t x2 = f2_fma(f2_pack(s[ch * 32 + 2 * i], s[ch * 32 + 2 * i + 1]), cc, mm);
+              float x0, x1, p0, p1;
+              f2_unpack(x2, x0, x1);
+              if (kEmu && emu_pair<C::EMU>(i)) {
+                f2_unpack(exp2_poly_x2(x0, x1), p0, p1);
+              } else {
+                p0 = ex2_approx(x0);
+                p1 = ex2_approx(x1);
+              }
+              const uint32_t b = pack_bf16x2(p0, p1);
+              pk[i] = b;
+              sf[i & 3] = f2_add(sf[i & 3], f2_pack(p0, p1));
+              if constexpr (!C::ONES)
+                sb[i & 3] = f2_add(sb[i & 3], f2_pack(__uint_as_float(b << 16),
+                                                      __uint_as_float(b & 0xFFFF0000u)));
+            }
+            tmem_st16(tS + ch * 16, pk);
+          }
+        };
+        if (C::EMU > 0 && j < n - 1) exps(std::true_type{});
+        else exps(std::false_type{});
       } else {
         // e4m3: four keys per 32-bit column, 256 p quantised; sb sums the quantised values
+        auto exps8 = [&](auto emu_tag) {
+          constexpr bool kEmu = decltype(emu_tag)::value;
 #pragma unroll
-        for (int ch = 0; ch < 2; ++ch) {
-          uint32_t pk[16];
+          for (int ch = 0; ch < 2; ++ch) {
+            uint32_t pk[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int k0 = ch * 64 + 4 * i;
-            float x0, x1, x2, x3;
-            f2_unpack(f2_fma(f2_pack(s[k0], s[k0 + 1]), cc, mm), x0, x1);
-            f2_unpack(f2_fma(f2_pack(s[k0 + 2], s[k0 + 3]), cc, mm), x2, x3);
-            const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-            const float p2 = ex2_approx(x2), p3 = ex2_approx(x3);
-            const uint32_t lo = pack_e4m3x2(kP8Scale * p0, kP8Scale * p1);
-            const uint32_t hi = pack_e4m3x2(kP8Scale * p2, kP8Scale * p3);
-            pk[i] = lo | (hi << 16);
-            float q0, q1, q2, q3;
-            unpack_e4m3x2(lo, q0, q1);
-            unpack_e4m3x2(hi, q2, q3);
-            sf[i & 3] = f2_add(sf[i & 3], f2_add(f2_pack(p0, p1), f2_pack(p2, p3)));
-            sb[i & 3] = f2_add(sb[i & 3], f2_add(f2_pack(q0, q1), f2_pack(q2, q3)));
+            for (int i = 0; i < 16; ++i) {
+              const int k0 = ch * 64 + 4 * i;
+              float x0, x1, x2, x3, p0, p1, p2, p3;
+              f2_unpack(f2_fma(f2_pack(s[k0], s[k0 + 1]), cc, mm), x0, x1);
+              f2_unpack(f2_fma(f2_pack(s[k0 + 2], s[k0 + 3]), cc, mm), x2, x3);
+              if (kEmu && emu_pair<C::EMU>(i)) {
+                f2_unpack(exp2_poly_x2(x0, x1), p0, p1);
+                f2_unpack(exp2_poly_x2(x2, x3), p2, p3);
+              } else {
+                p0 = ex2_approx(x0);
+                p1 = ex2_approx(x1);
+                p2 = ex2_approx(x2);
+                p3 = ex2_approx(x3);
+              }
+              const uint32_t lo = pack_e4m3x2(kP8Scale * p0, kP8Scale * p1);
+              const uint32_t hi = pack_e4m3x2(kP8Scale * p2, kP8Scale * p3);
+              pk[i] = lo | (hi << 16);
+              float q0, q1, q2, q3;
+              unpack_e4m3x2(lo, q0, q1);
+              unpack_e4m3x2(hi, q2, q3);
+              sf[i & 3] = f2_add(sf[i & 3], f2_add(f2_pack(p0, p1), f2_pack(p2, p3)));
+              sb[i & 3] = f2_add(sb[i & 3], f2_add(f2_pack(q0, q1), f2_pack(q2, q3)));
+            }
+            tmem_st16(tS + ch * 16, pk);
           }
-          tmem_st16(tS + ch * 16, pk);
-        }
+        };
+        if (C::EMU > 0 && j < n - 1) exps8(std::true_type{});
+        else exps8(std::false_type{});
       }
       {
         float a0, a1, b0, b1;
@@ -430,8 +511,16 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       if (ok) {
         tc_fence_after();
         // lb_run sums the weights the PV MMA used (for e4m3 in units of 1/256, which the
-        // division cancels); o_scale is 1, or the v descale.
-        const float inv = p.o_scale / lb_run;
+        // division cancels); with the ones columns that sum is O's column D.  o_scale is
+        // 1, or the v descale.
+        float wsum = lb_run;
+        if constexpr (C::ONES) {
+          uint32_t u[32];
+          tmem_ld32(tO + D, u);
+          tmem_wait_ld();
+          wsum = __uint_as_float(u[0]);
+        }
+        const float inv = p.o_scale / wsum;
         const bool valid = rpos < len;
         __nv_bfloat16* orow = p.o + (size_t(start + rpos) * p.Hq + h) * D;
 #pragma unroll 1

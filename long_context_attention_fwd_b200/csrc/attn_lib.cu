@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 
 #include <atomic>
+#include <chrono>
+#include <unistd.h>
 #include <cmath>
 #include <cstdint>
 #include <cstdio>
@@ -290,7 +292,7 @@ WsLayout ws_layout(int B, int Hq, long long T, int D) {
 // partial results.  (Measured on 16 x 16K-32K keys: 140 us with this plan, 161 us with
 // two CTAs per SM; on one 32K sequence: 34 us in one wave, 38 us in 1.7 waves.)
 constexpr int kPlanSMs = 148;
-int decode_max_parts() { return merge::kMaxStridedParts; }
+int decode_max_parts() { return decode::kMaxParts; }
 void decode_plan(int B, int Hkv, int Lmax, int* nsplit, int* tps) {
   const long long ntile = (Lmax + 127) / 128;
   const long long units = (long long)B * Hkv;
@@ -315,7 +317,7 @@ void decode_plan(int B, int Hkv, int Lmax, int* nsplit, int* tps) {
   *tps = int(t);
 }
 struct DecodeWs {
-  size_t o_part, lse_part, total;
+  size_t o_part, lse_part, ctr, total;
   int nsplit, tps, nparts;
 };
 DecodeWs decode_ws(int B, int Hq, int Hkv, int Lmax, int D) {
@@ -325,8 +327,28 @@ DecodeWs decode_ws(int B, int Hq, int Hkv, int Lmax, int D) {
   const size_t rows = size_t(B) * Hq;
   w.o_part = 0;
   w.lse_part = round_up(size_t(w.nparts) * rows * D * 2, 256);
-  w.total = w.lse_part + round_up(size_t(w.nparts) * rows * 4, 256);
+  w.ctr = w.lse_part + round_up(size_t(w.nparts) * rows * 4, 256);
+  w.total = w.ctr + round_up(size_t(B) * Hkv * 8, 256);
   return w;
+}
+
+// Tag of a decode call (48 bits, nonzero): the arrival words in the caller's workspace
+// count only arrivals that carry the current call's tag.  The sequence starts at a value
+// drawn from the clock and the process id, so that workspaces written by other processes
+// are unlikely to carry a live tag.
+unsigned long long next_decode_tag() {
+  static std::atomic<unsigned long long> ctr{0};
+  static const unsigned long long base = [] {
+    unsigned long long x = static_cast<unsigned long long>(
+        std::chrono::high_resolution_clock::now().time_since_epoch().count());
+    x ^= static_cast<unsigned long long>(getpid()) << 32;
+    x += 0x9E3779B97F4A7C15ull;  // SplitMix64 finaliser, to spread nearby seeds
+    x = (x ^ (x >> 30)) * 0xBF58476D1CE4E5B9ull;
+    x = (x ^ (x >> 27)) * 0x94D049BB133111EBull;
+    return x ^ (x >> 31);
+  }();
+  unsigned long long t = (base + ctr.fetch_add(1)) & ((1ull << 48) - 1);
+  return t ? t : 1;
 }
 attn_status check_decode_sizes(int B, int Hq, int Hkv, int Lmax, int D, float scale) {
   if (B < 1 || Hq < 1 || Hkv < 1 || Lmax < 1) return ATTN_ERR_INVALID_ARG;
@@ -552,9 +574,6 @@ attn_status attn_merge(const void* const* o_parts, const float* const* lse_parts
     p.o_parts[j] = nullptr;
     p.lse_parts[j] = nullptr;
   }
-  p.o_base = nullptr;
-  p.lse_base = nullptr;
-  p.o_stride = p.lse_stride = 0;
   if (!aligned(o, 16) || !aligned(lse, 4)) return ATTN_ERR_MISALIGNED;
   DeviceState* dev = nullptr;
   attn_status st = device_setup(&dev, o);
@@ -623,6 +642,10 @@ attn_status attn_decode(const void* q, const void* k_cache, const void* v_cache,
   p.nsplit = w.nsplit;
   p.tps = w.tps;
   p.rows = B * Hq;
+  p.ctr = reinterpret_cast<unsigned long long*>(ws + w.ctr);
+  p.tag = next_decode_tag();
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.status = dev->status;
   p.timeout_ns = g_timeout_ns.load();
@@ -633,32 +656,7 @@ attn_status attn_decode(const void* q, const void* k_cache, const void* v_cache,
     decode::attn_decode_kernel<64><<<unsigned(nblocks), decode::kThreads, decode::Cfg<64>::SMEM_ALLOC, s>>>(mq, mk, mv, p);
   else
     decode::attn_decode_kernel<128><<<unsigned(nblocks), decode::kThreads, decode::Cfg<128>::SMEM_ALLOC, s>>>(mq, mk, mv, p);
-  if ((st = check_launch("attn_decode_kernel launch")) != ATTN_OK) return st;
-
-  // Combine the 2 * nsplit partials of every (sequence, head) row exactly.
-  merge::Params mp;
-  for (int j = 0; j < merge::kMaxParts; ++j) {
-    mp.o_parts[j] = nullptr;
-    mp.lse_parts[j] = nullptr;
-  }
-  const unsigned rows = unsigned(B) * unsigned(Hq);
-  mp.o_base = reinterpret_cast<const uint4*>(ws + w.o_part);
-  mp.lse_base = reinterpret_cast<const float*>(ws + w.lse_part);
-  mp.o_stride = size_t(rows) * D * 2 / 16;
-  mp.lse_stride = rows;
-  mp.o = static_cast<uint4*>(o);
-  mp.lse = lse;
-  mp.nparts = w.nparts;
-  mp.H = 1;
-  mp.S = rows;
-  mp.rows = rows;
-  // One block per (sequence, head) row: the partials of a row are spread over the
-  // block's threads, so many splits do not serialise on one thread's loads.
-  if (D == 64)
-    merge::attn_merge_rows_kernel<64><<<rows, merge::kWideThreads, 0, s>>>(mp);
-  else
-    merge::attn_merge_rows_kernel<128><<<rows, merge::kWideThreads, 0, s>>>(mp);
-  return check_launch("attn_merge_kernel launch (decode)");
+  return check_launch("attn_decode_kernel launch");
 }
 
 attn_status attn_accumulate_bf16(float* acc, const void* x, long long n, int init, void* stream) {
@@ -814,6 +812,33 @@ extern "C" attn_status attn_selftest_umma_fp8(int mode, const void* a, const voi
   selftest::umma_selftest_fp8_kernel<<<1, 128, 2 * 128 * 128 + 2048, static_cast<cudaStream_t>(stream)>>>(
       ma, mb, mode, pin, pq, c, dev->status, g_timeout_ns.load());
   return check_launch("umma_selftest_fp8_kernel launch");
+}
+
+static __global__ void exp2_selftest_kernel(const float2* __restrict__ x, float2* __restrict__ y,
+                                            long long n2) {
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n2;
+       i += (long long)gridDim.x * blockDim.x) {
+    const float2 a = x[i];
+    float r0, r1;
+    f2_unpack(exp2_poly_x2(a.x, a.y), r0, r1);
+    y[i] = make_float2(r0, r1);
+  }
+}
+
+extern "C" attn_status attn_selftest_exp2(const float* x, float* y, long long n, void* stream) {
+  DeviceRestore restore_device;
+  if (!x || !y || n < 2 || (n & 1)) return ATTN_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(y, 16)) return ATTN_ERR_MISALIGNED;
+  DeviceState* dev = nullptr;
+  attn_status st = device_setup(&dev, x);
+  if (st != ATTN_OK) return st;
+  const long long n2 = n / 2;
+  const long long need = (n2 + 255) / 256;
+  const long long wave = (long long)dev->sms * 8;
+  exp2_selftest_kernel<<<unsigned(need < wave ? need : wave), 256, 0,
+                         static_cast<cudaStream_t>(stream)>>>(
+      reinterpret_cast<const float2*>(x), reinterpret_cast<float2*>(y), n2);
+  return check_launch("exp2_selftest_kernel launch");
 }
 
 // ------------------------------------------------------------------ backward without allocation

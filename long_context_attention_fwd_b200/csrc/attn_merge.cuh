@@ -31,17 +31,9 @@ namespace merge {
 constexpr int kMaxParts = 16;
 constexpr int kThreads = 256;
 
-constexpr int kMaxStridedParts = 256;
-
 struct Params {
   const uint4* o_parts[kMaxParts];    // [T][H][D] bf16 as groups of eight
   const float* lse_parts[kMaxParts];  // [B][H][S] fp32 (lse layout of the forward)
-  // Strided form (o_base != nullptr): partial j is o_base + j * o_stride and
-  // lse_base + j * lse_stride; used for the many per-split partials of decode.
-  const uint4* o_base;
-  const float* lse_base;
-  size_t o_stride;                    // in 16-byte units
-  size_t lse_stride;                  // in floats
   uint4* o;                           // [T][H][D] bf16
   float* lse;                         // [B][H][S]
   int nparts;
@@ -49,12 +41,8 @@ struct Params {
   unsigned rows;                      // T * H  (< 2^31, checked on the host)
 };
 
-__device__ __forceinline__ const uint4* part_o(const Params& p, int j) {
-  return p.o_base ? p.o_base + size_t(j) * p.o_stride : p.o_parts[j];
-}
-__device__ __forceinline__ const float* part_lse(const Params& p, int j) {
-  return p.lse_base ? p.lse_base + size_t(j) * p.lse_stride : p.lse_parts[j];
-}
+__device__ __forceinline__ const uint4* part_o(const Params& p, int j) { return p.o_parts[j]; }
+__device__ __forceinline__ const float* part_lse(const Params& p, int j) { return p.lse_parts[j]; }
 
 __device__ __forceinline__ void acc_bf16x8(float (&acc)[8], const uint4 x, const float w) {
   const uint32_t u[4] = {x.x, x.y, x.z, x.w};
@@ -161,70 +149,6 @@ __global__ void __launch_bounds__(kThreads) attn_merge_kernel(const __grid_const
       __stcs(p.o + off[k], y);
       if (c == 0) p.lse[li[k]] = lse_out[k];
     }
-  }
-}
-
-// Many partials of few rows (decode: up to 256 splits of B*Hq rows): one block per row,
-// kWideThreads threads = (D/8 column groups) x (part groups).  Each thread folds the
-// partials p = pg, pg + PG, ... of its column group with a running maximum; the part
-// groups are then combined through shared memory by the same log-sum-exp rule.  Strided
-// partials only; o and lse must not alias them.
-constexpr int kWideThreads = 256;
-
-template <int D>
-__global__ void __launch_bounds__(kWideThreads) attn_merge_rows_kernel(const __grid_constant__ Params p) {
-  constexpr int TPR = D / 8;
-  constexpr int PG = kWideThreads / TPR;
-  __shared__ float s_m[PG];
-  __shared__ float s_l[PG];
-  __shared__ float s_acc[PG][TPR][8];
-  const int c = threadIdx.x % TPR, pg = threadIdx.x / TPR;
-  const unsigned li = blockIdx.x;  // row: lse index (H = 1, S = rows)
-  const size_t off = size_t(li) * TPR + c;
-  float m = -INFINITY, l = 0.f, acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  for (int j = pg; j < p.nparts; j += PG) {
-    const float lj = part_lse(p, j)[li];
-    if (lj == -INFINITY) continue;
-    const uint4 x = __ldcs(part_o(p, j) + off);
-    if (lj > m) {                  // rescale what was folded so far to the new maximum
-      const float a = expf(m - lj);
-      l *= a;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) acc[e] *= a;
-      m = lj;
-    }
-    const float w = expf(lj - m);
-    l += w;
-    acc_bf16x8(acc, x, w);
-  }
-  if (c == 0) {
-    s_m[pg] = m;
-    s_l[pg] = l;
-  }
-  __syncthreads();
-  float mt = -INFINITY;
-#pragma unroll
-  for (int k = 0; k < PG; ++k) mt = fmaxf(mt, s_m[k]);
-  const float a = (m == -INFINITY) ? 0.f : expf(m - mt);
-#pragma unroll
-  for (int e = 0; e < 8; ++e) s_acc[pg][c][e] = acc[e] * a;
-  __syncthreads();
-  if (pg == 0) {
-    float lt = 0.f, o[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int k = 0; k < PG; ++k) {
-      if (s_m[k] != -INFINITY) lt += s_l[k] * expf(s_m[k] - mt);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) o[e] += s_acc[k][c][e];
-    }
-    const float inv = (mt == -INFINITY) ? 0.f : 1.f / lt;
-    uint4 y;
-    y.x = pack_bf16x2(o[0] * inv, o[1] * inv);
-    y.y = pack_bf16x2(o[2] * inv, o[3] * inv);
-    y.z = pack_bf16x2(o[4] * inv, o[5] * inv);
-    y.w = pack_bf16x2(o[6] * inv, o[7] * inv);
-    __stcs(p.o + off, y);
-    if (c == 0) p.lse[li] = (mt == -INFINITY) ? -INFINITY : mt + logf(lt);
   }
 }
 

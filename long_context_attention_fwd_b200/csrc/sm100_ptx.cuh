@@ -373,6 +373,28 @@ __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
   return d;
 }
 
+// 2^x for a pair of fp32 values on the FMA and integer pipes, leaving the MUFU unit to
+// other work.  x = j + f with j = rint(x) (adding and subtracting 1.5 * 2^23 rounds to
+// an integer and leaves j in the low bits of the sum), f in [-1/2, 1/2]; 2^f comes from
+// a degree-4 polynomial whose coefficients were fitted here by the Remez exchange on the
+// relative error over [-1/2, 1/2] (max relative error 2^-18.5 in fp32 Horner form), and
+// j is added into the exponent field.  x is clamped below at -125, so the result stays a
+// normal number: arguments below that give about 2^-125 instead of something smaller.
+__device__ __forceinline__ uint64_t exp2_poly_x2(float x0, float x1) {
+  const uint64_t x = f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+  const uint64_t rnd = f2_add(x, f2_pack(12582912.f, 12582912.f));
+  const uint64_t j = f2_add(rnd, f2_pack(-12582912.f, -12582912.f));
+  const uint64_t f = f2_fma(j, f2_pack(-1.f, -1.f), x);  // exact: |x - j| <= 1/2
+  uint64_t p = f2_fma(f2_pack(0.009570102f, 0.009570102f), f, f2_pack(0.05591786f, 0.05591786f));
+  p = f2_fma(p, f, f2_pack(0.24024744f, 0.24024744f));
+  p = f2_fma(p, f, f2_pack(0.69312179f, 0.69312179f));
+  p = f2_fma(p, f, f2_pack(0.99999928f, 0.99999928f));
+  // exponent: bits(rnd) = bits(1.5 * 2^23) + j, and bits(1.5 * 2^23) << 23 vanishes mod 2^32
+  const uint32_t r0 = uint32_t(rnd), r1 = uint32_t(rnd >> 32);
+  const uint32_t p0 = uint32_t(p), p1 = uint32_t(p >> 32);
+  return uint64_t((r0 << 23) + p0) | (uint64_t((r1 << 23) + p1) << 32);
+}
+
 // Packs two fp32 into bf16x2 (round to nearest even); `lo` goes to the low half.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;

@@ -89,3 +89,63 @@ def test_decode_deterministic():
     _, o1, l1 = _run(w)
     _, o2, l2 = _run(w)
     assert torch.equal(o1.view(torch.int16), o2.view(torch.int16)) and torch.equal(l1, l2)
+
+
+@pytest.mark.gpu
+def test_decode_workspace_needs_no_initialisation():
+    """The splits of a (sequence, kv head) count their arrivals in the workspace, and the
+    last one merges.  Whatever the workspace holds when a call starts (all ones, random
+    bytes, the previous call's leftovers) the result must be the same, bit for bit, and a
+    call leaves its arrival words cleared.  Replaying one captured launch (same call tag)
+    must also give the same result every time."""
+    from long_context_attention_fwd_b200 import ops
+    w = I.DecodeWorkload("decode_ws_reuse", B=3, Hq=28, Hkv=4, Lmax=2000, D=128,
+                         lens=[2000, 1, 777], seed=45)
+    x = I.make_decode_inputs(w, poison_tail=True)
+    q = torch_bf16(x["q"]).view(w.B, w.Hq, w.D)
+    k = torch_bf16(x["k"]).view(w.B, w.Lmax, w.Hkv, w.D)
+    v = torch_bf16(x["v"]).view(w.B, w.Lmax, w.Hkv, w.D)
+    cl = torch.from_numpy(x["cache_len"]).cuda()
+    nbytes = ops.attn_decode_workspace_size(q, k)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    ctr_bytes = -(-(w.B * w.Hkv * 8) // 256) * 256   # the arrival words end the workspace
+    outs = []
+    gen = torch.Generator(device="cuda").manual_seed(3)
+    for fill in ("ones", "random", "leftover", "leftover"):
+        if fill == "ones":
+            ws.fill_(0xFF)
+        elif fill == "random":
+            ws.copy_(torch.randint(0, 256, (nbytes,), generator=gen, device="cuda",
+                                   dtype=torch.int32).to(torch.uint8))
+        o = torch.full_like(q, float("nan"))
+        lse = torch.full((w.B, w.Hq), float("nan"), device="cuda")
+        ops.attn_decode(q, k, v, cl, scale=w.softmax_scale, out=o, lse=lse, workspace=ws)
+        torch.cuda.synchronize()
+        assert (ws[nbytes - ctr_bytes:nbytes - ctr_bytes + w.B * w.Hkv * 8] == 0).all(), fill
+        outs.append((o.clone(), lse.clone()))
+    _check(w, x, *outs[0])
+    for o, lse in outs[1:]:
+        assert torch.equal(o.view(torch.int16), outs[0][0].view(torch.int16))
+        assert torch.equal(lse, outs[0][1])
+    # one captured launch replayed: the call tag repeats, the cleared words make it work
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq), device="cuda")
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        ops.attn_decode(q, k, v, cl, scale=w.softmax_scale, out=o, lse=lse, workspace=ws)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, capture_error_mode="relaxed"):
+        ops.attn_decode(q, k, v, cl, scale=w.softmax_scale, out=o, lse=lse, workspace=ws)
+    for _ in range(3):
+        o.fill_(float("nan"))
+        graph.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(o.view(torch.int16), outs[0][0].view(torch.int16))
+        assert torch.equal(lse, outs[0][1])
+    del graph
+    from long_context_attention_fwd_b200 import capi
+    st, site = capi.attn_device_status(None)
+    assert st == capi.ATTN_OK, (capi.strerror(st), hex(site))

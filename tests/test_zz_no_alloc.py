@@ -10,7 +10,7 @@ failure has already run every other test."""
 import numpy as np
 import pytest
 
-from helpers import TOL_GRAD, bf16_ulp, make_case, rel_l2, torch_bf16
+from helpers import bf16_ulp, make_case, record, rel_l2, torch_bf16
 from long_context_attention_fwd_b200 import capi
 from long_context_attention_fwd_b200 import inputs as I
 
@@ -79,9 +79,13 @@ def test_noalloc_refuses_problems_larger_than_its_scratch():
 @pytest.mark.gpu
 @pytest.mark.parametrize("name,w", CASES, ids=[c[0] for c in CASES])
 def test_noalloc_matches_workspace_backward_on_consecutive_calls(name, w):
-    """dk and dv must equal the workspace backward's bit for bit (both are deterministic);
-    dq, summed with fp32 atomics in either, may differ only by the fp32 summation order:
-    at most one bf16 ulp per element."""
+    """dk and dv must equal the workspace backward's bit for bit (both are deterministic,
+    and both read the LSE and Delta rows the backward keeps in its scratch).  dq is summed
+    from per-key-tile partials with fp32 atomics in either run, so it may differ by the
+    summation order: the fp32 sums differ by a few fp32 roundings of the partials'
+    magnitudes (below 2^-14 of the tensor's largest element at these sizes), and the bf16
+    rounding of dq can turn that into one bf16 ulp.  A stale scratch (an accumulator not
+    cleared, rows of another call) would show up as errors of the order of dq itself."""
     from long_context_attention_fwd_b200 import ops
     q, k, v, do, cu, B, S = _tensors(w)
     scale = w.softmax_scale
@@ -106,6 +110,11 @@ def test_noalloc_matches_workspace_backward_on_consecutive_calls(name, w):
         assert torch.equal(dv, ref[2]), (call, "dv")
         g = dq.float().cpu().numpy().astype(np.float64)
         assert np.isfinite(g).all(), call
-        step = bf16_ulp(np.maximum(np.abs(g), np.abs(dq_ref)))
-        assert (np.abs(g - dq_ref) <= step).all(), (call, "dq")
-        assert rel_l2(g, dq_ref) <= TOL_GRAD, call
+        diff = np.abs(g - dq_ref)
+        bound = bf16_ulp(np.maximum(np.abs(g), np.abs(dq_ref))) + 2.0 ** -14 * np.abs(dq_ref).max()
+        e = rel_l2(g, dq_ref)
+        record(f"noalloc/{name}/call{call}", dq_max_abs_diff=float(diff.max()),
+               dq_n_differ=int((diff > 0).sum()), dq_rel_l2=e,
+               dq_worst_diff_over_bound=float((diff / bound).max()))
+        assert (diff <= bound).all(), (call, "dq")
+        assert e <= 1e-3, (call, e)
