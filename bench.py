@@ -494,7 +494,7 @@ def decode_measurements(dev, stream, peaks, reps=20):
             ts.append(e0.elapsed_time(e1))
         ms = statistics.median(ts)
         gbs = w.io_bytes() / (ms * 1e-3) / 1e9
-        out[w.name] = {"kernels": "attn_decode_kernel + attn_merge_kernel (strided)",
+        out[w.name] = {"kernels": "attn_decode_kernel (split-KV partials merged by the last split)",
                        "bound": "hbm", "ms": ms, "bytes": w.io_bytes(), "achieved": gbs,
                        "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
                        "tokens_per_s": w.B / (ms * 1e-3),
@@ -732,13 +732,29 @@ def run_gpu(args, w: I.Workload):
 def run_profile_case(args):
     """One launch of the forward and/or backward on a reduced synthetic problem, for ncu
     captures that must stay small (a few GB on the device, one launch of each kernel):
-    --profile B,Hq,Hkv,S,D [--profile-op fwd|bwd|both] [--profile-outliers].  Inputs are
+    --profile B,Hq,Hkv,S,D [--profile-op fwd|bwd|both|decode] [--profile-outliers]
+    (decode: B sequences of S cached keys, two decode steps).  Inputs are
     drawn on the GPU (N(0,1) * 0.5, or N(0,1) with 1% of q, k entries x8); the backward
     needs the forward's output, so --profile-op bwd also launches the forward once."""
     import torch
     from long_context_attention_fwd_b200 import capi, ops
     B, Hq, Hkv, S, D = (int(x) for x in args.profile.split(","))
     dev = torch.device("cuda", 0)
+    if args.profile_op == "decode":
+        # one decode step: B sequences of S cached keys each
+        g = torch.Generator(device=dev).manual_seed(20261203)
+        q = (torch.randn((B, Hq, D), generator=g, device=dev) * 0.5).bfloat16()
+        k = (torch.randn((B, S, Hkv, D), generator=g, device=dev) * 0.5).bfloat16()
+        v = (torch.randn((B, S, Hkv, D), generator=g, device=dev) * 0.5).bfloat16()
+        cl = torch.full((B,), S, dtype=torch.int32, device=dev)
+        for _ in range(2):
+            ops.attn_decode(q, k, v, cl)
+        torch.cuda.synchronize()
+        st, site = capi.attn_device_status(None)
+        if st != capi.ATTN_OK:
+            raise RuntimeError(f"device status {capi.strerror(st)} site={site:#x}")
+        print(json.dumps({"profile_case": [B, Hq, Hkv, S, D], "op": "decode", "status": "ok"}))
+        return 0
     g = torch.Generator(device=dev).manual_seed(20261203)
     mult = 1.0 if args.profile_outliers else 0.5
 
@@ -769,7 +785,7 @@ def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--profile", default=None, metavar="B,Hq,Hkv,S,D",
                     help="one launch on a reduced synthetic problem, for ncu captures")
-    ap.add_argument("--profile-op", default="both", choices=["fwd", "bwd", "both"])
+    ap.add_argument("--profile-op", default="both", choices=["fwd", "bwd", "both", "decode"])
     ap.add_argument("--profile-outliers", action="store_true")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)

@@ -136,8 +136,8 @@ attn_status attn_bwd_noalloc(const void* q, const void* k, const void* v, const 
                              const int32_t* cu_seqlens, void* stream);
 
 /* Bytes of device workspace attn_decode needs (0 for invalid sizes).  It holds the
- * per-split partial results, 2 * nsplit partials of B*Hq rows (bf16 o and fp32 lse) where
- * nsplit is fixed by (B, Hkv, Lmax), and one 8-byte arrival word per (sequence, kv head). */
+ * per-split partial results, nsplit partials of B*Hq rows (bf16 o and fp32 lse) where
+ * nsplit is fixed by (B, Hkv, Lmax), and one 8-byte done flag per split. */
 size_t attn_decode_workspace_size(int B, int Hq, int Hkv, int Lmax, int D);
 
 /* Decode attention over a key/value cache: one new query token per sequence attends to
@@ -154,11 +154,11 @@ size_t attn_decode_workspace_size(int B, int Hq, int Hkv, int Lmax, int D);
  *   - The cache is split along the keys; every split writes a partial (o, lse) into
  *     `workspace` (>= attn_decode_workspace_size bytes, 256-byte aligned, caller-owned),
  *     and the last split of each (sequence, kv head) to finish combines them exactly, in
- *     the same launch.  The splits count their arrivals in the workspace's arrival
- *     words; each word carries a 48-bit tag of the call, so the workspace needs no
- *     initialisation (leftover contents are taken for another call's, except with
- *     probability 2^-48 per word), and a call leaves its words cleared.  Two calls
- *     whose work overlaps on the GPU must not share a workspace.
+ *     the same launch.  Each split marks itself done with a flag word holding a 64-bit
+ *     tag of the call, so the workspace needs no initialisation (leftover contents count
+ *     as another call's, except with probability 2^-64 per word), and a call leaves its
+ *     flags cleared.  Two calls whose work overlaps on the GPU must not share a
+ *     workspace.
  *   - D in {64, 128}; Hq a multiple of Hkv with Hq/Hkv <= 128; B*Lmax and B*Hq < 2^31.
  *   - Pointers as in every entry point (16-byte aligned tensors, 4-byte lse/cache_len).
  *   - Deterministic. */

@@ -26,12 +26,15 @@
 // the rows of the last V tile past the length are zeroed in shared memory before its PV
 // product (whatever the cache holds there, 0 * NaN would otherwise poison O).
 //
-// The last CTA of a (sequence, kv head) to finish combines the partials of every split
-// into o and lse (the exact log-sum-exp rule of attn_merge), so a decode step is one
-// launch.  CTAs count their arrivals on a per-(sequence, kv head) word in the caller's
-// workspace, which may hold anything when the call starts: the word carries a 48-bit tag
-// of the call that wrote it, and a word with another tag counts as zero.  The merging CTA
-// clears its word again, so the next call (or a replay of the same launch) starts clean.
+// Each CTA first combines its two streams into one partial (o_s, lse_s).  The last CTA of
+// a (sequence, kv head) to finish then combines the partials of every split into o and
+// lse (the exact log-sum-exp rule of attn_merge), so a decode step is one launch.  The
+// CTAs find the last one without a counter: each writes a flag word carrying the call's
+// tag into the caller's workspace (which may hold anything when the call starts), fences,
+// and reads the flags of every split of its group; a CTA that sees them all tagged
+// merges.  With sequentially consistent fences at least one CTA sees all the others'
+// flags; when two do, both write the same result.  The merging CTA clears the flags, so
+// a replay of the same launch (same tag) starts clean.
 #pragma once
 #include <cuda_bf16.h>
 #include "attn_merge.cuh"
@@ -51,17 +54,17 @@ constexpr int kRegsCompute = 216;
 static_assert(128 * kRegsControl + 256 * kRegsCompute <= kThreads * kRegsLaunch, "register split");
 constexpr float kRescaleThreshold = 8.0f;
 constexpr int kSlab = 128 * 128;
-constexpr int kMaxParts = 256;  // partials per row: 2 streams x at most 128 splits
+constexpr int kMaxSplits = 128;  // splits (and partials) per (sequence, kv head)
 
 struct Params {
   const int32_t* cache_len;  // [B] (device); clamped to [0, Lmax]
-  __nv_bfloat16* o_part;     // [nparts][B*Hq][D], nparts = 2 * nsplit
-  float* lse_part;           // [nparts][B*Hq]
+  __nv_bfloat16* o_part;     // [nsplit][B*Hq][D]: one partial per split
+  float* lse_part;           // [nsplit][B*Hq]
   int Hq, G, Hkv, Lmax;
   int nsplit, tps;           // splits per (sequence, kv head); tiles per split
   int rows;                  // B * Hq (row stride between partials)
-  unsigned long long* ctr;   // [B * Hkv] arrival words (caller workspace, any initial value)
-  unsigned long long tag;    // this call's tag: nonzero, below 2^48
+  unsigned long long* flags; // [B * Hkv][nsplit] done flags (caller workspace, any initial value)
+  unsigned long long tag;    // this call's tag (nonzero)
   __nv_bfloat16* o;          // [B * Hq][D] result
   float* lse;                // [B * Hq]
   float scale_log2;
@@ -79,10 +82,11 @@ struct Cfg {
   static constexpr int OFF_V = OFF_K + NS * KV_BYTES;
   static constexpr int OFF_BAR = OFF_V + NS * KV_BYTES;
   // q_full, k_full[NS], k_empty[NS], v_full[NS], v_empty[NS], v_raw, s_full[2], p_full[2],
-  // o_final[2], drain
-  static constexpr int NBAR = 1 + 4 * NS + 1 + 7;
+  // o_final[2], drain, x_full
+  static constexpr int NBAR = 1 + 4 * NS + 1 + 8;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-  static constexpr int SMEM_BYTES = OFF_MISC + 16;
+  static constexpr int OFF_X = OFF_MISC + 16;    // stream 1's (m, l, lb) per row: 3 x 128 fp32
+  static constexpr int SMEM_BYTES = OFF_X + 3 * 128 * 4;
   static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O0 = 256, COL_O1 = 256 + D;
@@ -91,25 +95,8 @@ struct Cfg {
 enum : unsigned {
   kSiteKEmpty = 0x300, kSiteVEmpty, kSiteQFull, kSiteKFull, kSiteVFull, kSitePFull, kSiteSFull,
   kSiteOFinal, kSiteVRaw, kSiteDrainQ, kSiteDrainK, kSiteDrainV, kSiteDrainVRaw, kSiteDrainMMA,
-  kSiteTicket
+  kSiteXFull
 };
-
-// Counts this CTA's arrival on `word`: bits 63..16 hold the tag of the call that last
-// counted there, bits 15..0 its count.  A word with another tag (an earlier call, or
-// memory never written, which matches a given 48-bit tag with probability 2^-48) counts
-// as zero.  Returns the count including this arrival, or -1 if the compare-and-swap
-// loop gave up (it retries only while other CTAs of the same call arrive at once).
-__device__ __forceinline__ int arrive_count(unsigned long long* word, unsigned long long tag) {
-  unsigned long long cur = atomicAdd(word, 0ull);
-#pragma unroll 1
-  for (int i = 0; i < (1 << 16); ++i) {
-    const unsigned long long want = (cur >> 16) == tag ? cur + 1 : ((tag << 16) | 1ull);
-    const unsigned long long prev = atomicCAS(word, cur, want);
-    if (prev == cur) return int(want & 0xFFFFull);
-    cur = prev;
-  }
-  return -1;
-}
 
 // Combines the nparts partials of rows row0 .. row0 + G - 1 into p.o and p.lse, with all
 // kThreads threads of the CTA: LSE = ln sum_j exp(LSE_j), O = sum_j exp(LSE_j - LSE) O_j
@@ -218,6 +205,10 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   uint64_t* p_full = s_full + 2;
   uint64_t* o_final = p_full + 2;
   uint64_t* drain = o_final + 2;
+  uint64_t* x_full = drain + 1;    // stream 1's row statistics are in shared memory
+  float* x_m = reinterpret_cast<float*>(smem + C::OFF_X);
+  float* x_l = x_m + 128;
+  float* x_lb = x_l + 128;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   const int nw = (p.G + 31) >> 5;  // softmax warps per stream that own rows < G
@@ -238,6 +229,7 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       mbar_init(&o_final[t], 1);
     }
     mbar_init(drain, 1);
+    mbar_init(x_full, nw);
     fence_mbar_init();
   }
   if (warp == kWarpMMA) {
@@ -394,7 +386,7 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     const int qw = warp & 3;
     const int r = qw * 32 + lane;
     if (qw < nw) {
-      const int nt = n_t[t];
+      const int nt = t ? n_t[1] : n_t[0];
       const float c = p.scale_log2;
       const uint32_t colS = t ? C::COL_S1 : C::COL_S0;
       const uint32_t colO = t ? C::COL_O1 : C::COL_O0;
@@ -491,40 +483,69 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         __syncwarp();
         if (lane == 0) mbar_arrive(&p_full[t]);
       }
-      // Partial result of this stream: rows < G only.
-      const int part = 2 * s + t;
-      const bool valid = r < p.G;
-      __nv_bfloat16* orow = p.o_part + (size_t(part) * p.rows + row0 + r) * D;
-      float* lrow = p.lse_part + size_t(part) * p.rows + row0 + r;
-      if (nt == 0) {
-        if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(orow);
-#pragma unroll
-          for (int k = 0; k < D / 8; ++k) dst[k] = make_uint4(0u, 0u, 0u, 0u);
-          *lrow = -INFINITY;
-        }
-      } else if (ok) {
+      // One partial per split: stream 1 hands its row statistics to stream 0 through
+      // shared memory, and stream 0 combines both accumulators (each relative to its own
+      // running maximum) into o_s = (a0 O0 + a1 O1) / (a0 lb0 + a1 lb1) and
+      // lse_s = ln(a0 l0 + a1 l1) + M, with a_t = 2^(m_t - M), M = max(m0, m1).  A stream
+      // with no tile has m = -inf, weight 0, and its accumulator is never read.
+      if (ok && nt > 0) {
         ok = __all_sync(0xffffffffu, mbar_wait(&o_final[t], 0, wc, kSiteOFinal));
-        if (ok) {
-          tc_fence_after();
-          const float inv = 1.f / lb_run;
+        if (ok) tc_fence_after();
+      }
+      if (t == 1) {
+        if (r < 128) {
+          x_m[r] = m_run;
+          x_l[r] = l_run;
+          x_lb[r] = lb_run;
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(x_full);
+      } else {
+        ok = __all_sync(0xffffffffu, mbar_wait(x_full, 0, wc, kSiteXFull)) && ok;
+        tc_fence_after();
+        const bool valid = r < p.G;
+        __nv_bfloat16* orow = p.o_part + (size_t(s) * p.rows + row0 + r) * D;
+        float* lrow = p.lse_part + size_t(s) * p.rows + row0 + r;
+        const float m1 = x_m[r], l1 = x_l[r], lb1 = x_lb[r];
+        const float M = fmaxf(m_run, m1);
+        if (nt == 0 || M == -INFINITY) {
+          if (valid) {
+            uint4* dst = reinterpret_cast<uint4*>(orow);
+#pragma unroll
+            for (int k = 0; k < D / 8; ++k) dst[k] = make_uint4(0u, 0u, 0u, 0u);
+            *lrow = -INFINITY;
+          }
+        } else if (ok) {
+          const bool has1 = n_t[1] > 0;
+          const float a0 = ex2_approx(m_run - M);
+          const float a1 = has1 ? ex2_approx(m1 - M) : 0.f;
+          const float inv = 1.f / (a0 * lb_run + a1 * lb1);
+          const float w0 = a0 * inv, w1 = a1 * inv;
+          const uint32_t tO1 = tmem_addr(tmem, qw * 32, C::COL_O1);
 #pragma unroll 1
-          for (int ch = 0; ch < D / 32; ++ch) {
-            uint32_t u[32];
-            tmem_ld32(tO + ch * 32, u);
+          for (int ch = 0; ch < D / 16; ++ch) {
+            uint32_t u[16], u1[16];
+            tmem_ld16(tO + ch * 16, u);
+            if (has1) tmem_ld16(tO1 + ch * 16, u1);
             tmem_wait_ld();
-            uint32_t pk[16];
+            uint32_t pk[8];
 #pragma unroll
-            for (int k = 0; k < 16; ++k)
-              pk[k] = pack_bf16x2(__uint_as_float(u[2 * k]) * inv, __uint_as_float(u[2 * k + 1]) * inv);
+            for (int k = 0; k < 8; ++k) {
+              float e0 = __uint_as_float(u[2 * k]) * w0, e1 = __uint_as_float(u[2 * k + 1]) * w0;
+              if (has1) {
+                e0 = fmaf(__uint_as_float(u1[2 * k]), w1, e0);
+                e1 = fmaf(__uint_as_float(u1[2 * k + 1]), w1, e1);
+              }
+              pk[k] = pack_bf16x2(e0, e1);
+            }
             if (valid) {
-              uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
-#pragma unroll
-              for (int k = 0; k < 4; ++k)
-                dst[k] = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+              uint4* dst = reinterpret_cast<uint4*>(orow + ch * 16);
+              dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+              dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
             }
           }
-          if (valid) *lrow = (m_run + __log2f(l_run)) * 0.69314718055994530942f;
+          if (valid) *lrow = (M + __log2f(a0 * l_run + a1 * l1)) * 0.69314718055994530942f;
         }
       }
     }
@@ -532,7 +553,7 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   }
 
   // ---- teardown: every role has drained; release tensor memory.
-  __threadfence();  // this CTA's partials are visible device-wide before its arrival counts
+  if (warp < 4 && warp < nw) __threadfence();  // the partial's writers: visible before the flag
   tc_fence_before();
   __syncthreads();
   if (warp == kWarpMMA) {
@@ -540,21 +561,25 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
 
-  // ---- the last CTA of this (sequence, kv head) to arrive merges every split's partials.
-  volatile int* s_last = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);
-  if (threadIdx.x == 0) {
-    const int cnt = arrive_count(p.ctr + bg, p.tag);
-    if (cnt < 0) {
-      atomicOr(p.status, kStatusTimeout);
-      atomicCAS(p.status + 1, 0u, kSiteTicket);
+  // ---- done flag; the CTA that sees every split of its group done merges the partials.
+  volatile int* s_merge = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);
+  if (warp == 0) {
+    volatile unsigned long long* fl = p.flags + size_t(bg) * p.nsplit;
+    if (lane == 0) fl[s] = p.tag;
+    __syncwarp();
+    __threadfence();  // sequentially consistent: this flag is ordered before the reads below
+    bool all = true;
+    for (int i = lane; i < p.nsplit; i += 32) all = all && fl[i] == p.tag;
+    all = __all_sync(0xffffffffu, all);
+    if (all) {
+      for (int i = lane; i < p.nsplit; i += 32) fl[i] = 0ull;  // a replay starts clean
     }
-    *s_last = cnt == p.nsplit;
-    if (cnt == p.nsplit) atomicExch(p.ctr + bg, 0ull);  // clear for the next call
+    if (lane == 0) *s_merge = all;
   }
   __syncthreads();
-  if (*s_last) {
+  if (*s_merge) {
     __threadfence();
-    merge_rows<D>(p, row0, p.G, 2 * p.nsplit, smem + C::OFF_K);  // K/V stages are free now
+    merge_rows<D>(p, row0, p.G, p.nsplit, smem + C::OFF_K);  // K/V stages are free now
   }
 }
 

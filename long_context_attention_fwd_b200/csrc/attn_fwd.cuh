@@ -48,11 +48,12 @@ constexpr int BN = 128;                // keys per K/V tile
 constexpr int kThreads = 384;          // 12 warps; warps 10-11 only complete the control warpgroup
 constexpr int kWarpTMA = 8;
 constexpr int kWarpMMA = 9;
-// Register split (setmaxnreg), as in the backward kernel: 168 at launch, 72 for the
-// control warpgroup, 216 for the two softmax warpgroups (128*72 + 256*216 = 384*168).
+// Register split (setmaxnreg), as in the backward kernel: 168 at launch, 88 for the
+// control warpgroup (the producer and MMA loops carry the item loop's state), 208 for the
+// two softmax warpgroups (128*88 + 256*208 = 384*168); ptxas spills nothing at this split.
 constexpr int kRegsLaunch = 168;
-constexpr int kRegsControl = 72;
-constexpr int kRegsCompute = 216;
+constexpr int kRegsControl = 88;
+constexpr int kRegsCompute = 208;
 static_assert(128 * kRegsControl + 256 * kRegsCompute <= kThreads * kRegsLaunch, "register split");
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when max grows > 2^8
 constexpr int kSlab = 128 * 128;       // one 128-row x 64-column bf16 swizzled slab (16 KB)
@@ -76,6 +77,7 @@ struct Params {
   float scale_log2;                    // softmax scale * log2(e) (* q, k descale for e4m3)
   float o_scale;                       // 1, or the v descale for e4m3
   int nblk;                            // (T >> 8) + nseq: upper bound of 256-row blocks
+  int nitems;                          // nblk * Hq work items
   unsigned* status;
   unsigned long long timeout_ns;
 };
@@ -108,8 +110,9 @@ struct Cfg {
   static constexpr int OFF_V = OFF_K + NS * KV_BYTES;
   static constexpr int OFF_ONES = OFF_V + NS * KV_BYTES;  // 128 x 64 bf16 slab (ONES only)
   static constexpr int OFF_BAR = OFF_ONES + (ONES ? kSlab : 0);
-  // q_full, k_full[NS], k_empty[NS], v_full[NS], v_empty[NS], s_full[2], p_full[2], o_final[2], drain
-  static constexpr int NBAR = 1 + 4 * NS + 7;
+  // q_full, q_empty, k_full[NS], k_empty[NS], v_full[NS], v_empty[NS], s_full[2], p_full[2],
+  // o_final[2], drain
+  static constexpr int NBAR = 2 + 4 * NS + 7;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16;
   static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;  // slack for 1024-byte alignment
@@ -128,8 +131,42 @@ __device__ __forceinline__ constexpr bool emu_pair(int i) {
 // Wait-site codes reported in the status word when a wait times out.
 enum : unsigned {
   kSiteKEmpty = 0x100, kSiteVEmpty, kSiteQFull, kSiteKFull, kSiteVFull, kSitePFull, kSiteSFull,
-  kSiteOFinal
+  kSiteOFinal, kSiteQEmpty
 };
+
+// One work item: 256 query rows (two 128-row tiles) of one head of one sequence.
+struct Item {
+  int h, g, seq, start, len, q_row0, jmax;
+  int n_t[2];  // K/V tiles each query tile sees (0: the tile lies past the sequence end)
+};
+
+// The k-th item of this CTA.  Items are numbered longest causal block first, heads
+// fastest.  The grid is persistent (one CTA per SM, or fewer when there are fewer items):
+// CTA c takes items c, 2G-1-c, 2G+c, 4G-1-c, ... of a G-CTA grid -- rounds of G items in
+// alternating direction, so that over two rounds every CTA gets one of the longer and one
+// of the shorter blocks.  A grid of one CTA per item gives each CTA exactly one item.
+__device__ __forceinline__ int item_index(int k) {
+  const int G = int(gridDim.x), c = int(blockIdx.x);
+  return k * G + ((k & 1) ? G - 1 - c : c);
+}
+
+// Fills `it` for item w; false for an index in the slack after a sequence's last block.
+__device__ __forceinline__ bool item_at(const Params& p, int w, Item& it) {
+  it.h = w % p.Hq;
+  int mb;
+  if (!locate_block<8>(p.sv, p.nblk - 1 - w / p.Hq, it.seq, mb, it.start, it.len)) return false;
+  it.g = it.h / p.G;
+  it.q_row0 = mb * 256;
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const int r0 = it.q_row0 + BM * t;
+    if (r0 >= it.len) it.n_t[t] = 0;
+    else if (p.causal) it.n_t[t] = (min(r0 + BM - 1, it.len - 1) >> 7) + 1;
+    else it.n_t[t] = (it.len + BN - 1) >> 7;
+  }
+  it.jmax = max(it.n_t[0], it.n_t[1]);
+  return true;
+}
 
 template <int D, bool FP8 = false>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -143,26 +180,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---- work item: (sequence, head, 256-row block), longest causal blocks first.
-  const int h = blockIdx.x % p.Hq;
-  const int gblk = p.nblk - 1 - int(blockIdx.x / p.Hq);
-  int seq, mb, start, len;
-  if (!locate_block<8>(p.sv, gblk, seq, mb, start, len)) return;  // uniform: no work
-  const int g = h / p.G;
-  const int q_row0 = mb * 256;
-  int n_t[2];
-#pragma unroll
-  for (int t = 0; t < 2; ++t) {
-    const int r0 = q_row0 + BM * t;
-    if (r0 >= len) n_t[t] = 0;
-    else if (p.causal) n_t[t] = (min(r0 + BM - 1, len - 1) >> 7) + 1;
-    else n_t[t] = (len + BN - 1) >> 7;
-  }
-  const int jmax = max(n_t[0], n_t[1]);
-
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* q_full = bars;
-  uint64_t* k_full = bars + 1;
+  uint64_t* q_empty = bars + 1;    // the item's last S MMA has read the Q tiles
+  uint64_t* k_full = bars + 2;
   uint64_t* k_empty = k_full + C::NS;
   uint64_t* v_full = k_empty + C::NS;
   uint64_t* v_empty = v_full + C::NS;
@@ -176,6 +197,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   if (threadIdx.x == 0) {
     *abort_flag = 0;
     mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
     for (int i = 0; i < C::NS; ++i) {
       mbar_init(&k_full[i], 1);
       mbar_init(&k_empty[i], 1);
@@ -221,34 +243,47 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
    reg_dealloc<kRegsControl>();
    if (warp == kWarpTMA) {
     // ------------------------------------------------------------ producer
+    // Per item: the two Q tiles (once the previous item's last S MMA has read the
+    // buffer), then K_j / V_j into the ring, whose position carries over from item to
+    // item, so the next item's tiles load while this one finishes.
     if (lane == 0) {
-      int nk = 0, nv = 0;
-      const uint32_t qbytes = (n_t[0] > 0 ? C::QT_BYTES : 0) + (n_t[1] > 0 ? C::QT_BYTES : 0);
-      mbar_arrive_expect_tx(q_full, qbytes);
-      for (int t = 0; t < 2; ++t) {
-        if (n_t[t] == 0) continue;
-        for (int hf = 0; hf < C::SLABS; ++hf)
-          tma_load_3d(&tm_q, q_full, smem + C::OFF_Q + t * C::QT_BYTES + hf * kSlab,
-                      hf * (128 / C::ES), h, start + q_row0 + BM * t);
-      }
-      for (int j = 0; j < jmax; ++j) {
-        const int st = j % C::NS;
-        const uint32_t ph = (j / C::NS) & 1;
-        if (!mbar_wait(&k_empty[st], ph ^ 1, wc, kSiteKEmpty)) break;
-        mbar_arrive_expect_tx(&k_full[st], C::KV_BYTES);
-        for (int hf = 0; hf < C::SLABS; ++hf)
-          tma_load_3d(&tm_k, &k_full[st], smem + C::OFF_K + st * C::KV_BYTES + hf * kSlab,
-                      hf * (128 / C::ES), g, start + BN * j);
-        ++nk;
-        if (!mbar_wait(&v_empty[st], ph ^ 1, wc, kSiteVEmpty)) break;
-        mbar_arrive_expect_tx(&v_full[st], C::KV_BYTES);
-        for (int hf = 0; hf < C::SLABS; ++hf)
-          tma_load_3d(&tm_v, &v_full[st], smem + C::OFF_V + st * C::KV_BYTES + hf * kSlab,
-                      hf * (128 / C::ES), g, start + BN * j);
-        ++nv;
+      int nq = 0, nk = 0, nv = 0;  // Q loads, K tiles, V tiles issued
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        const int w = item_index(k);
+        if (w >= p.nitems) break;
+        Item it;
+        if (!item_at(p, w, it)) continue;
+        if (nq > 0 && !(ok = mbar_wait(q_empty, (nq - 1) & 1, wc, kSiteQEmpty))) break;
+        const uint32_t qbytes = (it.n_t[0] > 0 ? C::QT_BYTES : 0) + (it.n_t[1] > 0 ? C::QT_BYTES : 0);
+        mbar_arrive_expect_tx(q_full, qbytes);
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          if (it.n_t[t] == 0) continue;
+          for (int hf = 0; hf < C::SLABS; ++hf)
+            tma_load_3d(&tm_q, q_full, smem + C::OFF_Q + t * C::QT_BYTES + hf * kSlab,
+                        hf * (128 / C::ES), it.h, it.start + it.q_row0 + BM * t);
+        }
+        ++nq;
+        for (int j = 0; j < it.jmax; ++j) {
+          const int st = nk % C::NS;
+          const uint32_t ph = (nk / C::NS) & 1;
+          if (!(ok = mbar_wait(&k_empty[st], ph ^ 1, wc, kSiteKEmpty))) break;
+          mbar_arrive_expect_tx(&k_full[st], C::KV_BYTES);
+          for (int hf = 0; hf < C::SLABS; ++hf)
+            tma_load_3d(&tm_k, &k_full[st], smem + C::OFF_K + st * C::KV_BYTES + hf * kSlab,
+                        hf * (128 / C::ES), it.g, it.start + BN * j);
+          ++nk;
+          if (!(ok = mbar_wait(&v_empty[st], ph ^ 1, wc, kSiteVEmpty))) break;
+          mbar_arrive_expect_tx(&v_full[st], C::KV_BYTES);
+          for (int hf = 0; hf < C::SLABS; ++hf)
+            tma_load_3d(&tm_v, &v_full[st], smem + C::OFF_V + st * C::KV_BYTES + hf * kSlab,
+                        hf * (128 / C::ES), it.g, it.start + BN * j);
+          ++nv;
+        }
       }
       // Drain: every issued copy must land before shared memory is released.
-      mbar_drain(q_full, 0, drain_ns(abort_flag, p.timeout_ns));
+      if (nq) mbar_drain(q_full, (nq - 1) & 1, drain_ns(abort_flag, p.timeout_ns));
       for (int st = 0; st < C::NS; ++st) {
         const int ck = nk > st ? (nk - 1 - st) / C::NS + 1 : 0;
         const int cv = nv > st ? (nv - 1 - st) / C::NS + 1 : 0;
@@ -293,29 +328,48 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             mma_ts(tmem + colO[t], tmem + colS[t] + kk * 8, bdesc, idPV, (acc || kk > 0) ? 1u : 0u);
         }
       };
-      bool ok = mbar_wait(q_full, 0, wc, kSiteQFull) && mbar_wait(&k_full[0], 0, wc, kSiteKFull);
-      if (ok) {
+      // Phase counts carry over from item to item: nq items' Q tiles consumed, kv the
+      // ring position of the item's first K/V tile, pc[t] P tiles of query tile t used.
+      // A new item's first S overwrites the previous item's last P only after the PV
+      // that read it (MMAs complete in order); its first PV overwrites O only after the
+      // softmax warps signalled the new item's first P, which they do after their
+      // epilogue of the previous item has read O.
+      int nq = 0, kv = 0, pc[2] = {0, 0};
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        const int w = item_index(k);
+        if (w >= p.nitems) break;
+        Item it;
+        if (!item_at(p, w, it)) continue;
+        const int n_t[2] = {it.n_t[0], it.n_t[1]};
+        const int jmax = it.jmax;
+        if (!(ok = mbar_wait(q_full, nq & 1, wc, kSiteQFull))) break;
+        ++nq;
+        if (!(ok = mbar_wait(&k_full[kv % C::NS], (kv / C::NS) & 1, wc, kSiteKFull))) break;
         tc_fence_after();
+#pragma unroll
         for (int t = 0; t < 2; ++t)
           if (n_t[t] > 0) {
-            issue_S(t, 0);
+            issue_S(t, kv % C::NS);
             mma_commit(&s_full[t]);
           }
-        mma_commit(&k_empty[0]);
+        mma_commit(&k_empty[kv % C::NS]);
+        if (jmax == 1) mma_commit(q_empty);  // the item's last S has been issued
         for (int j = 0; j < jmax && ok; ++j) {
-          const int st = j % C::NS;
-          if (!(ok = mbar_wait(&v_full[st], (j / C::NS) & 1, wc, kSiteVFull))) break;
+          const int st = (kv + j) % C::NS;
+          if (!(ok = mbar_wait(&v_full[st], ((kv + j) / C::NS) & 1, wc, kSiteVFull))) break;
           tc_fence_after();
           if (j < n_t[0]) {
-            if (!(ok = mbar_wait(&p_full[0], j & 1, wc, kSitePFull))) break;
+            if (!(ok = mbar_wait(&p_full[0], pc[0] & 1, wc, kSitePFull))) break;
+            ++pc[0];
             tc_fence_after();
             issue_PV(0, st, j > 0);
             if (j == n_t[0] - 1) mma_commit(&o_final[0]);
           }
           const bool nxt = j + 1 < jmax;
-          const int st1 = (j + 1) % C::NS;
+          const int st1 = (kv + j + 1) % C::NS;
           if (nxt) {
-            if (!(ok = mbar_wait(&k_full[st1], ((j + 1) / C::NS) & 1, wc, kSiteKFull))) break;
+            if (!(ok = mbar_wait(&k_full[st1], ((kv + j + 1) / C::NS) & 1, wc, kSiteKFull))) break;
             tc_fence_after();
             if (j + 1 < n_t[0]) {
               issue_S(0, st1);
@@ -323,7 +377,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
           }
           if (j < n_t[1]) {
-            if (!(ok = mbar_wait(&p_full[1], j & 1, wc, kSitePFull))) break;
+            if (!(ok = mbar_wait(&p_full[1], pc[1] & 1, wc, kSitePFull))) break;
+            ++pc[1];
             tc_fence_after();
             issue_PV(1, st, j > 0);
             if (j == n_t[1] - 1) mma_commit(&o_final[1]);
@@ -335,8 +390,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
               mma_commit(&s_full[1]);
             }
             mma_commit(&k_empty[st1]);
+            if (j + 2 == jmax) mma_commit(q_empty);  // the item's last S has been issued
           }
         }
+        kv += jmax;
       }
       // Drain: all MMAs must finish before TMEM and shared memory are released.
       mma_commit(drain);
@@ -349,204 +406,215 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const int t = warp >> 2;
     const int qw = warp & 3;
     const int r = qw * 32 + lane;
-    const int rpos = q_row0 + BM * t + r;
-    const int n = n_t[t];
     const float c = p.scale_log2;
     const uint32_t colS = t ? C::COL_S1 : C::COL_S0;
     const uint32_t colO = t ? C::COL_O1 : C::COL_O0;
     const uint32_t tS = tmem_addr(tmem, qw * 32, colS);
     const uint32_t tO = tmem_addr(tmem, qw * 32, colO);
-    float m_run = -INFINITY;  // reference maximum (log2 units) the accumulator is scaled to
-    float l_run = 0.f;        // running normaliser relative to m_run (fp32 probabilities)
-    float lb_run = 0.f;       // the same over the bf16-rounded probabilities fed to PV
+    int sc = 0, oc = 0;  // S tiles and epilogues of this query tile so far (barrier phases)
     bool ok = true;
-    for (int j = 0; j < n; ++j) {
-      ok = __all_sync(0xffffffffu, mbar_wait(&s_full[t], j & 1, wc, kSiteSFull));
-      if (!ok) break;
-      tc_fence_after();
-      float s[128];
-      {
-        uint32_t u0[32], u1[32], u2[32], u3[32];
-        tmem_ld32(tS + 0, u0);
-        tmem_ld32(tS + 32, u1);
-        tmem_ld32(tS + 64, u2);
-        tmem_ld32(tS + 96, u3);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          s[i] = __uint_as_float(u0[i]);
-          s[32 + i] = __uint_as_float(u1[i]);
-          s[64 + i] = __uint_as_float(u2[i]);
-          s[96 + i] = __uint_as_float(u3[i]);
-        }
-      }
-      if (j == n - 1) {
-        // Last tile of the row's range: causal diagonal, or the sequence's key bound.
-        const int lim = p.causal ? rpos : (len - 1);
-        const int cmax = lim - BN * j;
-#pragma unroll
-        for (int i = 0; i < 128; ++i)
-          if (i > cmax) s[i] = -INFINITY;
-      }
-      float mx;
-      {
-        float m4[4] = {s[0], s[1], s[2], s[3]};
-#pragma unroll
-        for (int i = 4; i < 124; i += 8) {  // elements 4 .. 123
-          m4[0] = fmax3(m4[0], s[i], s[i + 4]);
-          m4[1] = fmax3(m4[1], s[i + 1], s[i + 5]);
-          m4[2] = fmax3(m4[2], s[i + 2], s[i + 6]);
-          m4[3] = fmax3(m4[3], s[i + 3], s[i + 7]);
-        }
-        m4[0] = fmax3(m4[0], s[124], s[125]);
-        m4[1] = fmax3(m4[1], s[126], s[127]);
-        mx = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]);
-      }
-      const float mx2 = mx * c;
-      const bool need = mx2 > m_run + (FP8 ? kRescaleThresholdFp8 : kRescaleThreshold);
-      const float m_new = need ? mx2 : m_run;
-      const float alpha = need ? ex2_approx(m_run - m_new) : 1.f;
-      if (j > 0 && __any_sync(0xffffffffu, need)) {
-        uint32_t u[32];
-#pragma unroll 1
-        for (int ch = 0; ch < (C::NPV + 31) / 32; ++ch) {  // O, and the row-sum columns
-          tmem_ld32(tO + ch * 32, u);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * alpha);
-          tmem_st32(tO + ch * 32, u);
-        }
-      }
-      l_run *= alpha;
-      lb_run *= alpha;
-      m_run = m_new;
-      const float mneg = (m_run == -INFINITY) ? 0.f : -m_run;
-      const uint64_t cc = f2_pack(c, c), mm = f2_pack(mneg, mneg);
-      // Two running sums: of the fp32 probabilities (for the log-sum-exp) and of
-      // their bf16 roundings (the values the PV MMA consumes), so that O is
-      // normalised by exactly the weights it was accumulated with.  With the ones
-      // columns the second sum comes out of the PV MMA instead.
-      uint64_t sf[4] = {0, 0, 0, 0}, sb[4] = {0, 0, 0, 0};
-      if constexpr (!FP8) {
-        // Tiles with no masked score hand a share of the exponentials to the FMA pipe.
-        auto exps = [&](auto emu_tag) {
-          constexpr bool kEmu = decltype(emu_tag)::value;
-#pragma unroll
-          for (int ch = 0; ch < 4; ++ch) {
-            uint32_t pk[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const uint64_t x2 = f2_fma(f2_pack(s[ch * 32 + 2 * i], s[ch * 32 + 2 * i + 1]), cc, mm);
-              float x0, x1, p0, p1;
-              f2_unpack(x2, x0, x1);
-              if (kEmu && emu_pair<C::EMU>(i)) {
-                f2_unpack(exp2_poly_x2(x0, x1), p0, p1);
-              } else {
-                p0 = ex2_approx(x0);
-                p1 = ex2_approx(x1);
-              }
-              const uint32_t b = pack_bf16x2(p0, p1);
-              pk[i] = b;
-              sf[i & 3] = f2_add(sf[i & 3], f2_pack(p0, p1));
-              if constexpr (!C::ONES)
-                sb[i & 3] = f2_add(sb[i & 3], f2_pack(__uint_as_float(b << 16),
-                                                      __uint_as_float(b & 0xFFFF0000u)));
-            }
-            tmem_st16(tS + ch * 16, pk);
-          }
-        };
-        if (C::EMU > 0 && j < n - 1) exps(std::true_type{});
-        else exps(std::false_type{});
-      } else {
-        // e4m3: four keys per 32-bit column, 256 p quantised; sb sums the quantised values
-        auto exps8 = [&](auto emu_tag) {
-          constexpr bool kEmu = decltype(emu_tag)::value;
-#pragma unroll
-          for (int ch = 0; ch < 2; ++ch) {
-            uint32_t pk[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const int k0 = ch * 64 + 4 * i;
-              float x0, x1, x2, x3, p0, p1, p2, p3;
-              f2_unpack(f2_fma(f2_pack(s[k0], s[k0 + 1]), cc, mm), x0, x1);
-              f2_unpack(f2_fma(f2_pack(s[k0 + 2], s[k0 + 3]), cc, mm), x2, x3);
-              if (kEmu && emu_pair<C::EMU>(i)) {
-                f2_unpack(exp2_poly_x2(x0, x1), p0, p1);
-                f2_unpack(exp2_poly_x2(x2, x3), p2, p3);
-              } else {
-                p0 = ex2_approx(x0);
-                p1 = ex2_approx(x1);
-                p2 = ex2_approx(x2);
-                p3 = ex2_approx(x3);
-              }
-              const uint32_t lo = pack_e4m3x2(kP8Scale * p0, kP8Scale * p1);
-              const uint32_t hi = pack_e4m3x2(kP8Scale * p2, kP8Scale * p3);
-              pk[i] = lo | (hi << 16);
-              float q0, q1, q2, q3;
-              unpack_e4m3x2(lo, q0, q1);
-              unpack_e4m3x2(hi, q2, q3);
-              sf[i & 3] = f2_add(sf[i & 3], f2_add(f2_pack(p0, p1), f2_pack(p2, p3)));
-              sb[i & 3] = f2_add(sb[i & 3], f2_add(f2_pack(q0, q1), f2_pack(q2, q3)));
-            }
-            tmem_st16(tS + ch * 16, pk);
-          }
-        };
-        if (C::EMU > 0 && j < n - 1) exps8(std::true_type{});
-        else exps8(std::false_type{});
-      }
-      {
-        float a0, a1, b0, b1;
-        f2_unpack(f2_add(f2_add(sf[0], sf[1]), f2_add(sf[2], sf[3])), a0, a1);
-        f2_unpack(f2_add(f2_add(sb[0], sb[1]), f2_add(sb[2], sb[3])), b0, b1);
-        l_run += a0 + a1;
-        lb_run += b0 + b1;
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[t]);
-    }
-    if (ok && n > 0) {
-      ok = __all_sync(0xffffffffu, mbar_wait(&o_final[t], 0, wc, kSiteOFinal));
-      if (ok) {
+    for (int k = 0; ok; ++k) {
+      const int w = item_index(k);
+      if (w >= p.nitems) break;
+      Item it;
+      if (!item_at(p, w, it)) continue;
+      const int n = t ? it.n_t[1] : it.n_t[0];
+      if (n == 0) continue;
+      const int rpos = it.q_row0 + BM * t + r;
+      const int len = it.len;
+      float m_run = -INFINITY;  // reference maximum (log2 units) the accumulator is scaled to
+      float l_run = 0.f;        // running normaliser relative to m_run (fp32 probabilities)
+      float lb_run = 0.f;       // the same over the bf16-rounded probabilities fed to PV
+      for (int j = 0; j < n; ++j) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&s_full[t], sc & 1, wc, kSiteSFull));
+        if (!ok) break;
+        ++sc;
         tc_fence_after();
-        // lb_run sums the weights the PV MMA used (for e4m3 in units of 1/256, which the
-        // division cancels); with the ones columns that sum is O's column D.  o_scale is
-        // 1, or the v descale.
-        float wsum = lb_run;
-        if constexpr (C::ONES) {
-          uint32_t u[32];
-          tmem_ld32(tO + D, u);
+        float s[128];
+        {
+          uint32_t u0[32], u1[32], u2[32], u3[32];
+          tmem_ld32(tS + 0, u0);
+          tmem_ld32(tS + 32, u1);
+          tmem_ld32(tS + 64, u2);
+          tmem_ld32(tS + 96, u3);
           tmem_wait_ld();
-          wsum = __uint_as_float(u[0]);
-        }
-        const float inv = p.o_scale / wsum;
-        const bool valid = rpos < len;
-        __nv_bfloat16* orow = p.o + (size_t(start + rpos) * p.Hq + h) * D;
-#pragma unroll 1
-        for (int ch = 0; ch < D / 32; ++ch) {
-          uint32_t u[32];
-          tmem_ld32(tO + ch * 32, u);
-          tmem_wait_ld();
-          uint32_t pk[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            pk[i] = pack_bf16x2(__uint_as_float(u[2 * i]) * inv, __uint_as_float(u[2 * i + 1]) * inv);
-          if (valid) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-              dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+          for (int i = 0; i < 32; ++i) {
+            s[i] = __uint_as_float(u0[i]);
+            s[32 + i] = __uint_as_float(u1[i]);
+            s[64 + i] = __uint_as_float(u2[i]);
+            s[96 + i] = __uint_as_float(u3[i]);
           }
         }
-        if (valid) {
-          const float lse = (m_run + __log2f(l_run)) * 0.69314718055994530942f;
-          const size_t li = p.sv.cu ? size_t(h) * p.T + start + rpos
-                                    : (size_t(seq) * p.Hq + h) * p.sv.S + rpos;
-          p.lse[li] = lse;
+        if (j == n - 1) {
+          // Last tile of the row's range: causal diagonal, or the sequence's key bound.
+          const int lim = p.causal ? rpos : (len - 1);
+          const int cmax = lim - BN * j;
+#pragma unroll
+          for (int i = 0; i < 128; ++i)
+            if (i > cmax) s[i] = -INFINITY;
+        }
+        float mx;
+        {
+          float m4[4] = {s[0], s[1], s[2], s[3]};
+#pragma unroll
+          for (int i = 4; i < 124; i += 8) {  // elements 4 .. 123
+            m4[0] = fmax3(m4[0], s[i], s[i + 4]);
+            m4[1] = fmax3(m4[1], s[i + 1], s[i + 5]);
+            m4[2] = fmax3(m4[2], s[i + 2], s[i + 6]);
+            m4[3] = fmax3(m4[3], s[i + 3], s[i + 7]);
+          }
+          m4[0] = fmax3(m4[0], s[124], s[125]);
+          m4[1] = fmax3(m4[1], s[126], s[127]);
+          mx = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]);
+        }
+        const float mx2 = mx * c;
+        const bool need = mx2 > m_run + (FP8 ? kRescaleThresholdFp8 : kRescaleThreshold);
+        const float m_new = need ? mx2 : m_run;
+        const float alpha = need ? ex2_approx(m_run - m_new) : 1.f;
+        if (j > 0 && __any_sync(0xffffffffu, need)) {
+          uint32_t u[32];
+#pragma unroll 1
+          for (int ch = 0; ch < (C::NPV + 31) / 32; ++ch) {  // O, and the row-sum columns
+            tmem_ld32(tO + ch * 32, u);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * alpha);
+            tmem_st32(tO + ch * 32, u);
+          }
+        }
+        l_run *= alpha;
+        lb_run *= alpha;
+        m_run = m_new;
+        const float mneg = (m_run == -INFINITY) ? 0.f : -m_run;
+        const uint64_t cc = f2_pack(c, c), mm = f2_pack(mneg, mneg);
+        // Two running sums: of the fp32 probabilities (for the log-sum-exp) and of
+        // their bf16 roundings (the values the PV MMA consumes), so that O is
+        // normalised by exactly the weights it was accumulated with.  With the ones
+        // columns the second sum comes out of the PV MMA instead.
+        uint64_t sf[4] = {0, 0, 0, 0}, sb[4] = {0, 0, 0, 0};
+        if constexpr (!FP8) {
+          // Tiles with no masked score hand a share of the exponentials to the FMA pipe.
+          auto exps = [&](auto emu_tag) {
+            constexpr bool kEmu = decltype(emu_tag)::value;
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) {
+              uint32_t pk[16];
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const uint64_t x2 = f2_fma(f2_pack(s[ch * 32 + 2 * i], s[ch * 32 + 2 * i + 1]), cc, mm);
+                float x0, x1, p0, p1;
+                f2_unpack(x2, x0, x1);
+                if (kEmu && emu_pair<C::EMU>(i)) {
+                  f2_unpack(exp2_poly_x2(x0, x1), p0, p1);
+                } else {
+                  p0 = ex2_approx(x0);
+                  p1 = ex2_approx(x1);
+                }
+                const uint32_t b = pack_bf16x2(p0, p1);
+                pk[i] = b;
+                sf[i & 3] = f2_add(sf[i & 3], f2_pack(p0, p1));
+                if constexpr (!C::ONES)
+                  sb[i & 3] = f2_add(sb[i & 3], f2_pack(__uint_as_float(b << 16),
+                                                        __uint_as_float(b & 0xFFFF0000u)));
+              }
+              tmem_st16(tS + ch * 16, pk);
+            }
+          };
+          if (C::EMU > 0 && j < n - 1) exps(std::true_type{});
+          else exps(std::false_type{});
+        } else {
+          // e4m3: four keys per 32-bit column, 256 p quantised; sb sums the quantised values
+          auto exps8 = [&](auto emu_tag) {
+            constexpr bool kEmu = decltype(emu_tag)::value;
+#pragma unroll
+            for (int ch = 0; ch < 2; ++ch) {
+              uint32_t pk[16];
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const int k0 = ch * 64 + 4 * i;
+                float x0, x1, x2, x3, p0, p1, p2, p3;
+                f2_unpack(f2_fma(f2_pack(s[k0], s[k0 + 1]), cc, mm), x0, x1);
+                f2_unpack(f2_fma(f2_pack(s[k0 + 2], s[k0 + 3]), cc, mm), x2, x3);
+                if (kEmu && emu_pair<C::EMU>(i)) {
+                  f2_unpack(exp2_poly_x2(x0, x1), p0, p1);
+                  f2_unpack(exp2_poly_x2(x2, x3), p2, p3);
+                } else {
+                  p0 = ex2_approx(x0);
+                  p1 = ex2_approx(x1);
+                  p2 = ex2_approx(x2);
+                  p3 = ex2_approx(x3);
+                }
+                const uint32_t lo = pack_e4m3x2(kP8Scale * p0, kP8Scale * p1);
+                const uint32_t hi = pack_e4m3x2(kP8Scale * p2, kP8Scale * p3);
+                pk[i] = lo | (hi << 16);
+                float q0, q1, q2, q3;
+                unpack_e4m3x2(lo, q0, q1);
+                unpack_e4m3x2(hi, q2, q3);
+                sf[i & 3] = f2_add(sf[i & 3], f2_add(f2_pack(p0, p1), f2_pack(p2, p3)));
+                sb[i & 3] = f2_add(sb[i & 3], f2_add(f2_pack(q0, q1), f2_pack(q2, q3)));
+              }
+              tmem_st16(tS + ch * 16, pk);
+            }
+          };
+          if (C::EMU > 0 && j < n - 1) exps8(std::true_type{});
+          else exps8(std::false_type{});
+        }
+        {
+          float a0, a1, b0, b1;
+          f2_unpack(f2_add(f2_add(sf[0], sf[1]), f2_add(sf[2], sf[3])), a0, a1);
+          f2_unpack(f2_add(f2_add(sb[0], sb[1]), f2_add(sb[2], sb[3])), b0, b1);
+          l_run += a0 + a1;
+          lb_run += b0 + b1;
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[t]);
+      }
+      if (ok) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&o_final[t], oc & 1, wc, kSiteOFinal));
+        ++oc;
+        if (ok) {
+          tc_fence_after();
+          // lb_run sums the weights the PV MMA used (for e4m3 in units of 1/256, which the
+          // division cancels); with the ones columns that sum is O's column D.  o_scale is
+          // 1, or the v descale.
+          float wsum = lb_run;
+          if constexpr (C::ONES) {
+            uint32_t u[32];
+            tmem_ld32(tO + D, u);
+            tmem_wait_ld();
+            wsum = __uint_as_float(u[0]);
+          }
+          const float inv = p.o_scale / wsum;
+          const bool valid = rpos < len;
+          __nv_bfloat16* orow = p.o + (size_t(it.start + rpos) * p.Hq + it.h) * D;
+#pragma unroll 1
+          for (int ch = 0; ch < D / 32; ++ch) {
+            uint32_t u[32];
+            tmem_ld32(tO + ch * 32, u);
+            tmem_wait_ld();
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              pk[i] = pack_bf16x2(__uint_as_float(u[2 * i]) * inv, __uint_as_float(u[2 * i + 1]) * inv);
+            if (valid) {
+              uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+            }
+          }
+          if (valid) {
+            const float lse = (m_run + __log2f(l_run)) * 0.69314718055994530942f;
+            const size_t li = p.sv.cu ? size_t(it.h) * p.T + it.start + rpos
+                                      : (size_t(it.seq) * p.Hq + it.h) * p.sv.S + rpos;
+            p.lse[li] = lse;
+          }
         }
       }
-    }
+    }  // items
   }
 
   // ---- teardown: every role has drained; release tensor memory.

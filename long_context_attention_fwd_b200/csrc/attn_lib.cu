@@ -269,6 +269,16 @@ attn_status check_sizes(int B, int Hq, int Hkv, int S, int D, float scale, bool 
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Grid of the forward kernel.  Dense batches: persistent, one CTA per SM (its shared
+// memory admits one), each taking a fixed share of the items -- their lengths are known
+// from the item index alone, so the alternating rounds balance them.  Packed batches:
+// one CTA per item, so that the hardware block scheduler balances lengths the host
+// cannot see (they sit in device memory).
+unsigned fwd_grid(unsigned nitems, unsigned sms, bool packed) {
+  if (packed) return nitems;
+  return nitems < sms ? nitems : sms;
+}
+
 struct WsLayout {
   size_t dq_acc, lse2, delta, total;
   int ntile;
@@ -288,11 +298,11 @@ WsLayout ws_layout(int B, int Hq, long long T, int D) {
 // CTAs per SM of a 148-SM B200 in total (one CTA is resident per SM, so later CTAs fill
 // the gaps that uneven sequence lengths leave), with at least four 128-key tiles per
 // split.  When that gives less than two waves, one exact wave is better: every CTA then
-// starts at once and no SM waits on a second round.  At most decode_max_parts()
+// starts at once and no SM waits on a second round.  At most decode_max_splits()
 // partial results.  (Measured on 16 x 16K-32K keys: 140 us with this plan, 161 us with
 // two CTAs per SM; on one 32K sequence: 34 us in one wave, 38 us in 1.7 waves.)
 constexpr int kPlanSMs = 148;
-int decode_max_parts() { return decode::kMaxParts; }
+int decode_max_splits() { return decode::kMaxSplits; }
 void decode_plan(int B, int Hkv, int Lmax, int* nsplit, int* tps) {
   const long long ntile = (Lmax + 127) / 128;
   const long long units = (long long)B * Hkv;
@@ -308,8 +318,8 @@ void decode_plan(int B, int Hkv, int Lmax, int* nsplit, int* tps) {
     if (t > ntile) t = ntile;
     ns = (ntile + t - 1) / t;
   }
-  if (2 * ns > decode_max_parts()) {
-    ns = decode_max_parts() / 2;
+  if (ns > decode_max_splits()) {
+    ns = decode_max_splits();
     t = (ntile + ns - 1) / ns;
     ns = (ntile + t - 1) / t;
   }
@@ -317,25 +327,25 @@ void decode_plan(int B, int Hkv, int Lmax, int* nsplit, int* tps) {
   *tps = int(t);
 }
 struct DecodeWs {
-  size_t o_part, lse_part, ctr, total;
+  size_t o_part, lse_part, flags, total;
   int nsplit, tps, nparts;
 };
 DecodeWs decode_ws(int B, int Hq, int Hkv, int Lmax, int D) {
   DecodeWs w;
   decode_plan(B, Hkv, Lmax, &w.nsplit, &w.tps);
-  w.nparts = 2 * w.nsplit;
+  w.nparts = w.nsplit;  // each split combines its two streams into one partial
   const size_t rows = size_t(B) * Hq;
   w.o_part = 0;
   w.lse_part = round_up(size_t(w.nparts) * rows * D * 2, 256);
-  w.ctr = w.lse_part + round_up(size_t(w.nparts) * rows * 4, 256);
-  w.total = w.ctr + round_up(size_t(B) * Hkv * 8, 256);
+  w.flags = w.lse_part + round_up(size_t(w.nparts) * rows * 4, 256);
+  w.total = w.flags + round_up(size_t(B) * Hkv * w.nsplit * 8, 256);
   return w;
 }
 
-// Tag of a decode call (48 bits, nonzero): the arrival words in the caller's workspace
-// count only arrivals that carry the current call's tag.  The sequence starts at a value
-// drawn from the clock and the process id, so that workspaces written by other processes
-// are unlikely to carry a live tag.
+// Tag of a decode call (64 bits, nonzero): a split's done flag counts only when it holds
+// the current call's tag.  The sequence starts at a value drawn from the clock and the
+// process id, so that workspaces written by other processes are unlikely to hold a live
+// tag.
 unsigned long long next_decode_tag() {
   static std::atomic<unsigned long long> ctr{0};
   static const unsigned long long base = [] {
@@ -347,7 +357,7 @@ unsigned long long next_decode_tag() {
     x = (x ^ (x >> 27)) * 0x94D049BB133111EBull;
     return x ^ (x >> 31);
   }();
-  unsigned long long t = (base + ctr.fetch_add(1)) & ((1ull << 48) - 1);
+  const unsigned long long t = base + ctr.fetch_add(1);
   return t ? t : 1;
 }
 attn_status check_decode_sizes(int B, int Hq, int Hkv, int Lmax, int D, float scale) {
@@ -418,9 +428,10 @@ attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float
   p.scale_log2 = scale * 1.4426950408889634f;
   p.o_scale = 1.f;
   p.nblk = int((T >> 8) + B);
+  p.nitems = p.nblk * Hq;
   p.status = dev->status;
   p.timeout_ns = g_timeout_ns.load();
-  const dim3 grid(unsigned(p.nblk) * unsigned(Hq));
+  const dim3 grid(fwd_grid(unsigned(p.nitems), dev->sms, cu_seqlens != nullptr));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (D == 64)
     fwd::attn_fwd_kernel<64><<<grid, fwd::kThreads, fwd::Cfg<64>::SMEM_ALLOC, s>>>(mq, mk, mv, p);
@@ -461,9 +472,10 @@ attn_status attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, f
   p.scale_log2 = scale * q_descale * k_descale * 1.4426950408889634f;
   p.o_scale = v_descale;
   p.nblk = int((T >> 8) + B);
+  p.nitems = p.nblk * Hq;
   p.status = dev->status;
   p.timeout_ns = g_timeout_ns.load();
-  const dim3 grid(unsigned(p.nblk) * unsigned(Hq));
+  const dim3 grid(fwd_grid(unsigned(p.nitems), dev->sms, cu_seqlens != nullptr));
   fwd::attn_fwd_kernel<128, true><<<grid, fwd::kThreads, fwd::Cfg<128, true>::SMEM_ALLOC,
                                     static_cast<cudaStream_t>(stream)>>>(mq, mk, mv, p);
   return check_launch("attn_fwd_kernel<fp8> launch");
@@ -642,7 +654,7 @@ attn_status attn_decode(const void* q, const void* k_cache, const void* v_cache,
   p.nsplit = w.nsplit;
   p.tps = w.tps;
   p.rows = B * Hq;
-  p.ctr = reinterpret_cast<unsigned long long*>(ws + w.ctr);
+  p.flags = reinterpret_cast<unsigned long long*>(ws + w.flags);
   p.tag = next_decode_tag();
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;

@@ -93,10 +93,10 @@ def test_decode_deterministic():
 
 @pytest.mark.gpu
 def test_decode_workspace_needs_no_initialisation():
-    """The splits of a (sequence, kv head) count their arrivals in the workspace, and the
-    last one merges.  Whatever the workspace holds when a call starts (all ones, random
-    bytes, the previous call's leftovers) the result must be the same, bit for bit, and a
-    call leaves its arrival words cleared.  Replaying one captured launch (same call tag)
+    """The splits of a (sequence, kv head) mark themselves done in the workspace, and one
+    that sees them all done merges.  Whatever the workspace holds when a call starts (all
+    ones, random bytes, the previous call's leftovers) the result must be the same, bit for
+    bit, and a call leaves its done flags cleared.  Replaying one captured launch (same call tag)
     must also give the same result every time."""
     from long_context_attention_fwd_b200 import ops
     w = I.DecodeWorkload("decode_ws_reuse", B=3, Hq=28, Hkv=4, Lmax=2000, D=128,
@@ -108,7 +108,13 @@ def test_decode_workspace_needs_no_initialisation():
     cl = torch.from_numpy(x["cache_len"]).cuda()
     nbytes = ops.attn_decode_workspace_size(q, k)
     ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
-    ctr_bytes = -(-(w.B * w.Hkv * 8) // 256) * 256   # the arrival words end the workspace
+    # the workspace is nsplit bf16 partials, their fp32 lse rows, then one 8-byte done flag
+    # per (sequence, kv head, split), each part rounded up to 256 bytes; find nsplit
+    up = lambda x: -(-x // 256) * 256
+    rows = w.B * w.Hq
+    nsplit = next(n for n in range(1, 129)
+                  if up(n * rows * w.D * 2) + up(n * rows * 4) + up(w.B * w.Hkv * n * 8) == nbytes)
+    flag_at, flag_bytes = nbytes - up(w.B * w.Hkv * nsplit * 8), w.B * w.Hkv * nsplit * 8
     outs = []
     gen = torch.Generator(device="cuda").manual_seed(3)
     for fill in ("ones", "random", "leftover", "leftover"):
@@ -121,7 +127,7 @@ def test_decode_workspace_needs_no_initialisation():
         lse = torch.full((w.B, w.Hq), float("nan"), device="cuda")
         ops.attn_decode(q, k, v, cl, scale=w.softmax_scale, out=o, lse=lse, workspace=ws)
         torch.cuda.synchronize()
-        assert (ws[nbytes - ctr_bytes:nbytes - ctr_bytes + w.B * w.Hkv * 8] == 0).all(), fill
+        assert (ws[flag_at:flag_at + flag_bytes] == 0).all(), fill
         outs.append((o.clone(), lse.clone()))
     _check(w, x, *outs[0])
     for o, lse in outs[1:]:
