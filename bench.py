@@ -732,8 +732,9 @@ def run_gpu(args, w: I.Workload):
 def run_profile_case(args):
     """One launch of the forward and/or backward on a reduced synthetic problem, for ncu
     captures that must stay small (a few GB on the device, one launch of each kernel):
-    --profile B,Hq,Hkv,S,D [--profile-op fwd|bwd|both|decode] [--profile-outliers]
-    (decode: B sequences of S cached keys, two decode steps).  Inputs are
+    --profile B,Hq,Hkv,S,D [--profile-op fwd|fwd8|bwd|both|decode] [--profile-outliers]
+    (fwd8: two e4m3 forward launches after one bf16 one; decode: B sequences of S cached
+    keys, two decode steps).  Inputs are
     drawn on the GPU (N(0,1) * 0.5, or N(0,1) with 1% of q, k entries x8); the backward
     needs the forward's output, so --profile-op bwd also launches the forward once."""
     import torch
@@ -768,6 +769,14 @@ def run_profile_case(args):
     v, do = draw(Hkv, False), draw(Hq, False)
     scale = D ** -0.5
     o, lse = ops.attn_fwd(q, k, v, causal=True, scale=scale)
+    if args.profile_op == "fwd8":
+        # the e4m3 forward on the same inputs quantised per tensor (descale = max|x| / 448)
+        def q8(t):
+            d = float(t.abs().max().float()) / 448.0
+            return (t.float() / d).clamp_(-448.0, 448.0).to(torch.float8_e4m3fn), d
+        (q8_, qd), (k8_, kd), (v8_, vd) = q8(q), q8(k), q8(v)
+        for _ in range(2):
+            ops.attn_fwd_fp8(q8_, k8_, v8_, qd, kd, vd, causal=True, scale=scale, out=o, lse=lse)
     if args.profile_op in ("fwd", "both"):
         ops.attn_fwd(q, k, v, causal=True, scale=scale, out=o, lse=lse)
     if args.profile_op in ("bwd", "both"):
@@ -785,7 +794,7 @@ def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--profile", default=None, metavar="B,Hq,Hkv,S,D",
                     help="one launch on a reduced synthetic problem, for ncu captures")
-    ap.add_argument("--profile-op", default="both", choices=["fwd", "bwd", "both", "decode"])
+    ap.add_argument("--profile-op", default="both", choices=["fwd", "fwd8", "bwd", "both", "decode"])
     ap.add_argument("--profile-outliers", action="store_true")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
