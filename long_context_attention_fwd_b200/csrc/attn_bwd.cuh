@@ -16,10 +16,11 @@
 //   attn_bwd_kernel KV-stationary: one CTA holds a 128-key tile of one kv head (K, V in
 //                   shared memory, dK/dV accumulators in TMEM) and loops over the query
 //                   heads of its group and the 128-row query tiles that see it.
-//                   Per query tile: S^T = K Q^T, dP^T = V dO^T, dV += P^T dO,
-//                   dK += dS^T Q (P^T, dS^T read from TMEM as bf16), dQ_tile = dS K
-//                   (dS staged in shared memory), and dQ_tile is reduced into the fp32
-//                   accumulator with coalesced vector reductions.  dK/dV stay deterministic.
+//                   Per query tile: S^T = K Q^T, dP^T = V dO^T, dV += P^T dO (P^T read
+//                   from TMEM as bf16), dK += dS^T Q and dQ_tile = dS K (both reading the
+//                   one bf16 dS buffer in shared memory, K-major and MN-major), and dQ_tile
+//                   is reduced into the fp32 accumulator with coalesced vector reductions.
+//                   dK/dV stay deterministic.
 //   dq_convert      dq = bf16(scale * accumulator).
 //
 // Warps: 0-3 and 4-7 compute P^T and dS^T (one thread per key row; warps 0-3 take query
@@ -47,6 +48,12 @@ constexpr int kRegsControl = 72;
 constexpr int kRegsCompute = 144;
 static_assert(128 * kRegsControl + 384 * kRegsCompute <= kThreads * kRegsLaunch, "register split");
 constexpr int kSlab = 128 * 128;
+// The P/dS warpgroups hand dS over in four chunks of 32 query columns (1), so that the dK
+// MMA runs while the later chunks are computed, or all at once (0).
+#ifndef ATTN_BWD_DSCHUNK
+#define ATTN_BWD_DSCHUNK 1
+#endif
+constexpr int kDsChunks = ATTN_BWD_DSCHUNK ? 4 : 1;
 
 struct Params {
   SeqView sv;
@@ -75,9 +82,9 @@ struct Cfg {
   static constexpr int OFF_LSE = OFF_DS + 128 * 128 * 2;  // 2 stages x 128 fp32
   static constexpr int OFF_DELTA = OFF_LSE + 2 * 512;
   static constexpr int OFF_BAR = OFF_DELTA + 2 * 512;
-  // kv_full, q_full[2], q_empty[2], do_full[2], do_empty[2], s_full, dp_full, p_full, ds_full,
-  // dq_full, dq_free, dkv_final, drain
-  static constexpr int NBAR = 17;
+  // kv_full, q_full[2], q_empty[2], do_full[2], do_empty[2], s_full, dp_full, p_full,
+  // dq_full, dq_free, dkv_final, drain, ds_full[kDsChunks]
+  static constexpr int NBAR = 16 + kDsChunks;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16;
   static constexpr int kMaxDyn = 232448;
@@ -235,11 +242,11 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   uint64_t* s_full = bars + 9;
   uint64_t* dp_full = bars + 10;
   uint64_t* p_full = bars + 11;
-  uint64_t* ds_full = bars + 12;
-  uint64_t* dq_full = bars + 13;
-  uint64_t* dq_free = bars + 14;   // dQ columns of TMEM read out
-  uint64_t* dkv_final = bars + 15;
-  uint64_t* drain = bars + 16;
+  uint64_t* dq_full = bars + 12;
+  uint64_t* dq_free = bars + 13;   // dQ columns of TMEM read out
+  uint64_t* dkv_final = bars + 14;
+  uint64_t* drain = bars + 15;
+  uint64_t* ds_full = bars + 16;   // [kDsChunks] chunk c of dS is in shared memory
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   float* lse_s = reinterpret_cast<float*>(smem + C::OFF_LSE);
@@ -257,7 +264,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     mbar_init(s_full, 1);
     mbar_init(dp_full, 1);
     mbar_init(p_full, 8);
-    mbar_init(ds_full, 8);
+    for (int c = 0; c < kDsChunks; ++c) mbar_init(&ds_full[c], kDsChunks == 1 ? 8 : 4);
     mbar_init(dq_full, 1);
     mbar_init(dq_free, 4);
     mbar_init(dkv_final, 1);
@@ -341,8 +348,8 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         issue_T(C::COL_S, kb, smem_u32(smem + C::OFF_Q));
         mma_commit(s_full);
       }
-      // P^T and dS^T halves sit in TMEM columns [0, 32) and [96, 128) of their regions
-      // (warps 0-3 / warps 4-7, bf16 pairs): A-operand column of 16-row step kk.
+      // P^T halves sit in TMEM columns [0, 32) and [96, 128) of the S^T region (warps 0-3 /
+      // warps 4-7, bf16 pairs): A-operand column of 16-row step kk.
       auto a_col = [](int kk) -> uint32_t { return kk < 4 ? kk * 8 : 96 + (kk - 4) * 8; };
       // Per query tile: dP^T first (it needs neither P nor dS, so the dS step can start as
       // soon as P is done), then dV, the next S^T, dK and dQ.
@@ -369,12 +376,21 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           issue_T(C::COL_S, kb, smem_u32(smem + C::OFF_Q + (st ^ 1) * C::TILE));  // next S^T
           mma_commit(s_full);
         }
-        if (!(ok = mbar_wait(ds_full, it & 1, wc, kSiteDsFull))) break;
-        tc_fence_after();
+        // dK += dS^T Q (dS^T K-major in shared memory), chunk by chunk as dS arrives:
+        // chunk c covers query K steps 2c, 2c + 1 (warpgroup c / 2, local half c % 2).  The
+        // two warpgroups run side by side, so their first halves are taken first.
+        for (int j = 0; j < kDsChunks && ok; ++j) {
+          const int c = kDsChunks == 4 ? ((j & 1) << 1) | (j >> 1) : 0;
+          if (!(ok = mbar_wait(&ds_full[c], it & 1, wc, kSiteDsFull))) break;
+          tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)  // dK += dS^T Q
-          mma_ts(tmem + C::COL_DK, tmem + C::COL_DP + a_col(kk), sdesc_sw128(qb + kk * 2048, kSlab, 1024),
-                 idKV, (it > 0 || kk > 0) ? 1u : 0u);
+          for (int k2 = 0; k2 < 8 / kDsChunks; ++k2) {
+            const int kk = c * (8 / kDsChunks) + k2;
+            mma_ss(tmem + C::COL_DK, sdesc_sw128(dsb + (kk >> 2) * kSlab + (kk & 3) * 32, 16, 1024),
+                   sdesc_sw128(qb + kk * 2048, kSlab, 1024), idKV, (it > 0 || kk > 0) ? 1u : 0u);
+          }
+        }
+        if (!ok) break;
         mma_commit(&q_empty[st]);
         if (!C::DQ_ALIAS && it > 0 && !(ok = mbar_wait(dq_free, (it - 1) & 1, wc, kSiteDqFree))) break;
         tc_fence_after();
@@ -392,10 +408,10 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     reg_alloc<kRegsCompute>();
     // ------------------------------------------------------------ P^T and dS^T
     // Warpgroup wg takes query columns cb .. cb+63 of the tile (cb = 64 wg); thread r owns
-    // key row r.  The bf16 results are stored in place, packed two per 32-bit column, each
-    // inside the columns its own warpgroup reads: P^T over S^T columns cb + 32 wg ..
-    // + 31 (0-31 and 96-127), dS^T likewise over the dP^T columns.  So neither warpgroup
-    // overwrites a column the other has yet to read.
+    // key row r.  P^T is stored in place as bf16, packed two per 32-bit column, inside the
+    // columns its own warpgroup reads: S^T columns cb + 32 wg .. + 31 (0-31 and 96-127),
+    // so neither warpgroup overwrites a column the other has yet to read.  dS^T goes to
+    // shared memory only.
     const int wg = warp >> 2;
     const int qw = warp & 3;
     const int cb = wg * 64;
@@ -406,7 +422,6 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const uint32_t tS = tmem_addr(tmem, qw * 32, C::COL_S + cb);
     const uint32_t tPst = tmem_addr(tmem, qw * 32, C::COL_S + cb + 32 * wg);
     const uint32_t tP = tmem_addr(tmem, qw * 32, C::COL_DP + cb);
-    const uint32_t tDSst = tmem_addr(tmem, qw * 32, C::COL_DP + cb + 32 * wg);
     uint8_t* ds_row = smem + C::OFF_DS + wg * 16384 + (r >> 3) * 1024 + (r & 7) * 128;
     bool ok = true;
     for (int it = 0; it < iters; ++it) {
@@ -466,16 +481,14 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full);
 
-      // dS^T = P^T * (dP^T - Delta): written in place into the dP columns (bf16) for the
-      // dK MMA and into shared memory (MN-major) for the dQ MMA, once the previous dQ MMA
-      // has finished reading that buffer.
+      // dS^T = P^T * (dP^T - Delta), written as bf16 into shared memory once the previous
+      // dQ MMA has finished reading that buffer.  The one buffer is the A operand of both
+      // MMAs that use dS: MN-major dS for dQ = dS K, K-major dS^T for dK += dS^T Q.
       ok = __all_sync(0xffffffffu, mbar_wait(dp_full, it & 1, wc, kSiteDpFull) &&
                                        (it == 0 || mbar_wait(dq_full, (it - 1) & 1, wc, kSiteDqFull)));
       if (!ok) break;
       tc_fence_after();
       // dP^T in two halves: the second loads while the first half's dS^T is computed.
-      // That half's TMEM store waits for the load, since warpgroup 1 stores dS^T over
-      // the columns of dP^T's second half.
       uint32_t u[64];
       auto half_p = [&](int hf) -> uint32_t(&)[32] {
         return *reinterpret_cast<uint32_t(*)[32]>(u + 32 * hf);
@@ -483,7 +496,6 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       tmem_ld32(tP + 0, half_p(0));
       tmem_wait_ld_regs(half_p(0));
       tmem_ld32(tP + 32, half_p(1));
-      uint32_t pk_first[16];
 #pragma unroll
       for (int ch = 0; ch < 2; ++ch) {
         if (ch == 1) tmem_wait_ld_regs(half_p(1));
@@ -503,13 +515,6 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           pk[2 * i4] = pack_bf16x2(a0, a1);
           pk[2 * i4 + 1] = pack_bf16x2(a2, a3);
         }
-        if (ch == 0) {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) pk_first[i] = pk[i];
-        } else {
-          tmem_st16(tDSst, pk_first);
-          tmem_st16(tDSst + 16, pk);
-        }
         // shared memory: this warpgroup's 64 query rows are 64-row block wg; local rows
         // ch*32 .. ch*32+31 are 16-byte chunks ch*4 .. ch*4+3 of the key row's line
 #pragma unroll
@@ -518,12 +523,22 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           *reinterpret_cast<uint4*>(ds_row + ((chunk ^ (r & 7)) << 4)) =
               make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
         }
+        if (kDsChunks == 4) {
+          // The dK MMA may read this chunk now.  The last chunk also orders both halves'
+          // TMEM loads before the hand-over, since the dQ MMA (after every chunk) writes
+          // over the dP^T columns at D = 128.
+          fence_async_smem();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&ds_full[wg * 2 + ch]);
+        }
       }
-      fence_async_smem();
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(ds_full);
+      if (kDsChunks == 1) {
+        fence_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ds_full[0]);
+      }
     }
     // epilogue: dV rows (warps 0-3), dK rows scaled (warps 4-7)
     if (ok) {

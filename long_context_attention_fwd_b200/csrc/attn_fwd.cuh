@@ -22,12 +22,16 @@
 // other tile's PV and the next S, so MMA and exponentials overlap.
 //
 // The exponentials and the MMAs of a tile take about equally long at D = 128, and the
-// exponentials twice as long at D = 64, so the MUFU unit paces the loop.  Two changes
-// take work off it and off the softmax threads:
-//   - a share of the exponentials (Cfg::EMU pairs of every 16) is evaluated by a
-//     polynomial on the FMA pipe (exp2_poly_x2) in tiles without masked scores;
-//   - at D = 64 the normaliser over the bf16 weights comes out of the PV MMA itself, as
-//     16 extra accumulator columns against a column of ones in shared memory.
+// exponentials twice as long at D = 64, so the softmax chain paces the loop.  At D = 64
+// two changes take work off the softmax threads and start the PV product sooner:
+//   - the normaliser over the bf16 weights comes out of the PV MMA itself, as 16 extra
+//     accumulator columns against a column of ones in shared memory;
+//   - P is handed to the MMA warp in four chunks of 32 keys, so the PV MMAs of the first
+//     keys run while the later ones are exponentiated (at D = 128 the extra barrier
+//     round trips cost more than the overlap gains, so P goes over as one tile there).
+// A share of the exponentials (Cfg::EMU pairs of every 16, in tiles without masked
+// scores) can also be evaluated by a polynomial on the FMA pipe (exp2_poly_x2); the share
+// is 0 by default, since no share measured faster at either head dim.
 //
 // FP8 = true is the e4m3 variant (D = 128): Q, K, V are e4m3 with per-tensor descale
 // factors folded into the softmax scale (q, k) and the epilogue (v); the MMAs are
@@ -62,10 +66,22 @@ constexpr int kSlab = 128 * 128;       // one 128-row x 64-column bf16 swizzled 
 #define ATTN_FWD_EMU64 0
 #endif
 #ifndef ATTN_FWD_EMU128
-#define ATTN_FWD_EMU128 2
+#define ATTN_FWD_EMU128 0
 #endif
 #ifndef ATTN_FWD_EMU_FP8
 #define ATTN_FWD_EMU_FP8 0
+#endif
+// The softmax warps hand P to the MMA warp in chunks (1), so that a tile's PV product
+// starts on the first keys while the later ones are still being exponentiated, or as
+// one tile (0), per head dim.
+#ifndef ATTN_FWD_PCHUNK64
+#define ATTN_FWD_PCHUNK64 1
+#endif
+#ifndef ATTN_FWD_PCHUNK128
+#define ATTN_FWD_PCHUNK128 0
+#endif
+#ifndef ATTN_FWD_PCHUNK_FP8
+#define ATTN_FWD_PCHUNK_FP8 1
 #endif
 
 struct Params {
@@ -103,6 +119,9 @@ struct Cfg {
   static constexpr int SLABS = D * ES / 128;             // 128-byte swizzle rows per tile row
   static constexpr int KSTEPS = D * ES / 32;             // MMAs over D (32 bytes of K each)
   static constexpr int PSTEPS = BN * ES / 32;            // MMAs over the keys of a tile
+  static constexpr int SMCH = FP8 ? 2 : 4;               // softmax chunks of 16 P columns
+  static constexpr int PCH =                              // P hand-overs per tile
+      (FP8 ? ATTN_FWD_PCHUNK_FP8 : (D == 64 ? ATTN_FWD_PCHUNK64 : ATTN_FWD_PCHUNK128)) ? SMCH : 1;
   static constexpr int QT_BYTES = BM * D * ES;
   static constexpr int KV_BYTES = BN * D * ES;
   static constexpr int OFF_Q = 0;
@@ -110,9 +129,9 @@ struct Cfg {
   static constexpr int OFF_V = OFF_K + NS * KV_BYTES;
   static constexpr int OFF_ONES = OFF_V + NS * KV_BYTES;  // 128 x 64 bf16 slab (ONES only)
   static constexpr int OFF_BAR = OFF_ONES + (ONES ? kSlab : 0);
-  // q_full, q_empty, k_full[NS], k_empty[NS], v_full[NS], v_empty[NS], s_full[2], p_full[2],
-  // o_final[2], drain
-  static constexpr int NBAR = 2 + 4 * NS + 7;
+  // q_full, q_empty, k_full[NS], k_empty[NS], v_full[NS], v_empty[NS], s_full[2],
+  // p_full[2][PCH], o_final[2], drain
+  static constexpr int NBAR = 2 + 4 * NS + 5 + 2 * PCH;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16;
   static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;  // slack for 1024-byte alignment
@@ -188,8 +207,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   uint64_t* v_full = k_empty + C::NS;
   uint64_t* v_empty = v_full + C::NS;
   uint64_t* s_full = v_empty + C::NS;
-  uint64_t* p_full = s_full + 2;
-  uint64_t* o_final = p_full + 2;
+  uint64_t* p_full = s_full + 2;           // [2][PCH]: chunk c of tile t's P is in TMEM
+  uint64_t* o_final = p_full + 2 * C::PCH;
   uint64_t* drain = o_final + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
@@ -206,7 +225,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&s_full[t], 1);
-      mbar_init(&p_full[t], 4);
+      for (int c = 0; c < C::PCH; ++c) mbar_init(&p_full[t * C::PCH + c], 4);
       mbar_init(&o_final[t], 1);
     }
     mbar_init(drain, 1);
@@ -312,21 +331,31 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                    sdesc_sw128(kb + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
         }
       };
-      auto issue_PV = [&](int t, int st, bool acc) {
+      // O_t (+)= P_t V over the tile's keys, chunk by chunk as the softmax warps hand the
+      // chunks of P over (parity `ph` of this tile's hand-overs); false if a wait failed.
+      auto issue_PV = [&](int t, int st, bool acc, uint32_t ph) -> bool {
         const uint32_t vb = smem_u32(smem + C::OFF_V + st * C::KV_BYTES);
         // MN-major V: 64-element N blocks kSlab apart; with the ones columns the second
         // N block is the ones slab, which lies after every V stage.
         constexpr uint32_t kLbo0 = C::ONES ? uint32_t(C::OFF_ONES - C::OFF_V) : uint32_t(kSlab);
         const uint32_t lbo = C::ONES ? kLbo0 - uint32_t(st * C::KV_BYTES) : kLbo0;
+        constexpr int KPC = C::PSTEPS / C::PCH;  // K steps per hand-over
 #pragma unroll
-        for (int kk = 0; kk < C::PSTEPS; ++kk) {
-          // K step: 32 bytes of keys = 32 / ES key rows of 128 bytes in the MN-major V tile
-          const uint64_t bdesc = sdesc_sw128(vb + kk * (4096 / C::ES), lbo, 1024);
-          if constexpr (FP8)
-            mma_ts_f8(tmem + colO[t], tmem + colS[t] + kk * 8, bdesc, idPV, (acc || kk > 0) ? 1u : 0u);
-          else
-            mma_ts(tmem + colO[t], tmem + colS[t] + kk * 8, bdesc, idPV, (acc || kk > 0) ? 1u : 0u);
+        for (int c = 0; c < C::PCH; ++c) {
+          if (!mbar_wait(&p_full[t * C::PCH + c], ph, wc, kSitePFull)) return false;
+          tc_fence_after();
+#pragma unroll
+          for (int k2 = 0; k2 < KPC; ++k2) {
+            const int kk = c * KPC + k2;
+            // K step: 32 bytes of keys = 32 / ES key rows of 128 bytes in the MN-major V tile
+            const uint64_t bdesc = sdesc_sw128(vb + kk * (4096 / C::ES), lbo, 1024);
+            if constexpr (FP8)
+              mma_ts_f8(tmem + colO[t], tmem + colS[t] + kk * 8, bdesc, idPV, (acc || kk > 0) ? 1u : 0u);
+            else
+              mma_ts(tmem + colO[t], tmem + colS[t] + kk * 8, bdesc, idPV, (acc || kk > 0) ? 1u : 0u);
+          }
         }
+        return true;
       };
       // Phase counts carry over from item to item: nq items' Q tiles consumed, kv the
       // ring position of the item's first K/V tile, pc[t] P tiles of query tile t used.
@@ -360,10 +389,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           if (!(ok = mbar_wait(&v_full[st], ((kv + j) / C::NS) & 1, wc, kSiteVFull))) break;
           tc_fence_after();
           if (j < n_t[0]) {
-            if (!(ok = mbar_wait(&p_full[0], pc[0] & 1, wc, kSitePFull))) break;
+            if (!(ok = issue_PV(0, st, j > 0, pc[0] & 1))) break;
             ++pc[0];
-            tc_fence_after();
-            issue_PV(0, st, j > 0);
             if (j == n_t[0] - 1) mma_commit(&o_final[0]);
           }
           const bool nxt = j + 1 < jmax;
@@ -377,10 +404,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
           }
           if (j < n_t[1]) {
-            if (!(ok = mbar_wait(&p_full[1], pc[1] & 1, wc, kSitePFull))) break;
+            if (!(ok = issue_PV(1, st, j > 0, pc[1] & 1))) break;
             ++pc[1];
-            tc_fence_after();
-            issue_PV(1, st, j > 0);
             if (j == n_t[1] - 1) mma_commit(&o_final[1]);
           }
           mma_commit(&v_empty[st]);
@@ -493,6 +518,16 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // normalised by exactly the weights it was accumulated with.  With the ones
         // columns the second sum comes out of the PV MMA instead.
         uint64_t sf[4] = {0, 0, 0, 0}, sb[4] = {0, 0, 0, 0};
+        // Hands chunk ch of P to the MMA warp once its TMEM stores have completed (after
+        // every chunk, or after the last one when P goes over as one tile).
+        auto publish = [&](int ch) {
+          constexpr int per = C::SMCH / C::PCH;
+          if ((ch + 1) % per != 0) return;
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&p_full[t * C::PCH + ch / per]);
+        };
         if constexpr (!FP8) {
           // Tiles with no masked score hand a share of the exponentials to the FMA pipe.
           auto exps = [&](auto emu_tag) {
@@ -519,6 +554,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                                                         __uint_as_float(b & 0xFFFF0000u)));
               }
               tmem_st16(tS + ch * 16, pk);
+              publish(ch);
             }
           };
           if (C::EMU > 0 && j < n - 1) exps(std::true_type{});
@@ -555,6 +591,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 sb[i & 3] = f2_add(sb[i & 3], f2_add(f2_pack(q0, q1), f2_pack(q2, q3)));
               }
               tmem_st16(tS + ch * 16, pk);
+              publish(ch);
             }
           };
           if (C::EMU > 0 && j < n - 1) exps8(std::true_type{});
@@ -567,10 +604,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           l_run += a0 + a1;
           lb_run += b0 + b1;
         }
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&p_full[t]);
       }
       if (ok) {
         ok = __all_sync(0xffffffffu, mbar_wait(&o_final[t], oc & 1, wc, kSiteOFinal));
