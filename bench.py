@@ -52,8 +52,11 @@ def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         d = json.load(open(p))
+        d["_source"] = "MEASURED_PEAKS.json"
         return d, "measured (MEASURED_PEAKS.json)"
-    return dict(FALLBACK_PEAKS), "fallback (no MEASURED_PEAKS.json)"
+    d = dict(FALLBACK_PEAKS)
+    d["_source"] = "fallback peaks (no MEASURED_PEAKS.json)"
+    return d, "fallback (no MEASURED_PEAKS.json)"
 
 
 def dist_env():
@@ -89,14 +92,18 @@ def max_over_ranks(values, device):
 
 
 # ---------------------------------------------------------------- ncu traffic
-KERNEL_SOURCES = ("sm100_ptx.cuh", "attn_common.cuh", "attn_fwd.cuh", "attn_bwd.cuh",
-                  "attn_merge.cuh")
+# The sources each kernel is compiled from: a traffic record is valid only for these bytes.
+KERNEL_SOURCES = {
+    "attn_fwd_kernel": ("sm100_ptx.cuh", "attn_common.cuh", "attn_fwd.cuh"),
+    "attn_bwd_kernel": ("sm100_ptx.cuh", "attn_common.cuh", "attn_bwd.cuh"),
+    "attn_merge_kernel_4parts": ("sm100_ptx.cuh", "attn_merge.cuh"),
+}
 
 
-def kernel_sources_sha1() -> str:
+def kernel_sources_sha1(kernel: str) -> str:
     import hashlib
     h = hashlib.sha1()
-    for name in KERNEL_SOURCES:
+    for name in KERNEL_SOURCES[kernel]:
         with open(os.path.join(ROOT, "long_context_attention_fwd_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()
@@ -104,13 +111,13 @@ def kernel_sources_sha1() -> str:
 
 def measured_traffic(workload: str, kernel: str):
     """DRAM bytes (read + write) per launch of `kernel` from the ncu capture summarised
-    in profiles/traffic.json, or None when the kernel sources changed since the capture."""
+    in profiles/traffic.json, or None when the kernel's sources changed since the capture."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
-        d = json.load(open(path))
-        if d.get("kernel_sources_sha1") != kernel_sources_sha1():
+        rec = json.load(open(path))["workloads"][workload][kernel]
+        if rec.get("sources_sha1") != kernel_sources_sha1(kernel):
             return None
-        return d["workloads"][workload][kernel]["dram_bytes_per_launch"]
+        return rec["dram_bytes_per_launch"]
     except Exception:
         return None
 
@@ -350,7 +357,7 @@ def ring_measurements(wr: I.Workload, q, k, v, o, lse, stream, peaks, world=4, r
                   "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
                   "traffic": (measured_traffic(wr.name, "attn_merge_kernel_4parts")
                               if world == 4 else None),
-                  "peak_source": "MEASURED_PEAKS.json hbm_gbs (copy, read+write bytes)"},
+                  "peak_source": f"{peaks['_source']} hbm_gbs (copy, read+write bytes)"},
         "ring_fwd_one_gpu": {"world": world, "ms": ring_ms,
                              "tflops": I.flop_fwd(wr) / (ring_ms * 1e-3) / 1e12,
                              "single_kernel_fwd_ms": fwd_ms, "attn_fwd_launches": n_fwd,
@@ -411,7 +418,7 @@ def ulysses_measurements(wr: I.Workload, q, k, v, do, stream, peaks, world=4, re
                                  f"groups [{world}, {B * S}, {Hq // world}, {D}]",
                      "ms": tr_ms, "bytes_per_launch": tr_bytes, "achieved": gbs, "peak": hbm,
                      "unit": "GB/s", "frac": gbs / hbm,
-                     "peak_source": "MEASURED_PEAKS.json hbm_gbs (copy, read+write bytes)"},
+                     "peak_source": f"{peaks['_source']} hbm_gbs (copy, read+write bytes)"},
         "ulysses_fwd_bwd_one_gpu": {
             "world": world, "ms": uly_ms,
             "tflops": (I.flop_fwd(wr) + I.flop_bwd(wr)) / (uly_ms * 1e-3) / 1e12,
@@ -455,7 +462,7 @@ def fp8_measurements(wr: I.Workload, q, k, v, stream, peaks, reps=10):
     peak = 2.0 * float(peaks.get("bf16_tflops"))
     return {"kernel": "attn_fwd_kernel<128, e4m3>", "bound": "tensor", "ms": fp8_ms,
             "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
-            "peak_source": "MEASURED_PEAKS.json bf16_tflops (burst) x 2, the nominal fp8:bf16 ratio",
+            "peak_source": f"{peaks['_source']} bf16_tflops (burst) x 2, the nominal fp8:bf16 ratio",
             "bf16_fwd_ms_same_run": bf16_ms, "speedup_vs_bf16": bf16_ms / fp8_ms,
             "inputs": "the bench workload's q, k, v quantised per tensor to e4m3 on the GPU"}
 

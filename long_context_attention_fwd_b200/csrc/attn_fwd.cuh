@@ -74,6 +74,16 @@ constexpr int kSlab = 128 * 128;       // one 128-row x 64-column bf16 swizzled 
 // The softmax warps hand P to the MMA warp in chunks (1), so that a tile's PV product
 // starts on the first keys while the later ones are still being exponentiated, or as
 // one tile (0), per head dim.
+// Row sums of the rounded weights by mixed-precision adds (bf16 or f16 operand, fp32
+// accumulator) instead of unpacking to fp32 first (1), or by unpacking (0).
+#ifndef ATTN_FWD_MIXADD
+#define ATTN_FWD_MIXADD 1
+#endif
+// e4m3: the factor 256 of P = e4m3(256 p) folded into the exponent, exp2(x + 8) (1), or
+// applied by a multiply (0).
+#ifndef ATTN_FWD_FP8FOLD
+#define ATTN_FWD_FP8FOLD 1
+#endif
 #ifndef ATTN_FWD_PCHUNK64
 #define ATTN_FWD_PCHUNK64 1
 #endif
@@ -139,6 +149,26 @@ struct Cfg {
   static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O0 = 256, COL_O1 = ONES ? 384 : 256 + D;
   static_assert(COL_O1 + NPV <= TMEM_COLS, "TMEM budget");
 };
+
+// a += low bf16 of v, b += high bf16 of v: each bf16 taken exactly, one fp32 rounding per add
+// (mixed-precision add, no unpacking).
+__device__ __forceinline__ void add_bf16x2_f32(uint32_t v, float& a, float& b) {
+  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+      "add.rn.f32.bf16 %0, lo, %0;\n\tadd.rn.f32.bf16 %1, hi, %1;\n\t}"
+      : "+f"(a), "+f"(b) : "r"(v));
+}
+// The same for two f16 values.
+__device__ __forceinline__ void add_f16x2_f32(uint32_t v, float& a, float& b) {
+  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+      "add.rn.f32.f16 %0, lo, %0;\n\tadd.rn.f32.f16 %1, hi, %1;\n\t}"
+      : "+f"(a), "+f"(b) : "r"(v));
+}
+// The two e4m3 values of the low 16 bits of `v`, exactly, as an f16x2 (low byte in the low half).
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t v) {
+  uint32_t h2;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(uint16_t(v & 0xFFFFu)));
+  return h2;
+}
 
 // Pair i (0..15) of a 32-score chunk is exponentiated on the FMA pipe when this holds:
 // EMU of every 16 pairs, spread evenly.
@@ -513,11 +543,15 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         m_run = m_new;
         const float mneg = (m_run == -INFINITY) ? 0.f : -m_run;
         const uint64_t cc = f2_pack(c, c), mm = f2_pack(mneg, mneg);
+        // e4m3: exp2(x + 8) = 256 exp2(x), the scaled weight that is quantised
+        constexpr float kFold = (FP8 && ATTN_FWD_FP8FOLD) ? 8.0f : 0.0f;
+        const uint64_t mm8 = f2_pack(mneg + kFold, mneg + kFold);
         // Two running sums: of the fp32 probabilities (for the log-sum-exp) and of
         // their bf16 roundings (the values the PV MMA consumes), so that O is
         // normalised by exactly the weights it was accumulated with.  With the ones
         // columns the second sum comes out of the PV MMA instead.
         uint64_t sf[4] = {0, 0, 0, 0}, sb[4] = {0, 0, 0, 0};
+        float sbf[4] = {0.f, 0.f, 0.f, 0.f};  // the rounded weights' sum, mixed-precision adds
         // Hands chunk ch of P to the MMA warp once its TMEM stores have completed (after
         // every chunk, or after the last one when P goes over as one tile).
         auto publish = [&](int ch) {
@@ -549,9 +583,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const uint32_t b = pack_bf16x2(p0, p1);
                 pk[i] = b;
                 sf[i & 3] = f2_add(sf[i & 3], f2_pack(p0, p1));
-                if constexpr (!C::ONES)
-                  sb[i & 3] = f2_add(sb[i & 3], f2_pack(__uint_as_float(b << 16),
-                                                        __uint_as_float(b & 0xFFFF0000u)));
+                if constexpr (!C::ONES) {
+                  if constexpr (ATTN_FWD_MIXADD)
+                    add_bf16x2_f32(b, sbf[(i & 1) * 2], sbf[(i & 1) * 2 + 1]);
+                  else
+                    sb[i & 3] = f2_add(sb[i & 3], f2_pack(__uint_as_float(b << 16),
+                                                          __uint_as_float(b & 0xFFFF0000u)));
+                }
               }
               tmem_st16(tS + ch * 16, pk);
               publish(ch);
@@ -570,8 +608,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
               for (int i = 0; i < 16; ++i) {
                 const int k0 = ch * 64 + 4 * i;
                 float x0, x1, x2, x3, p0, p1, p2, p3;
-                f2_unpack(f2_fma(f2_pack(s[k0], s[k0 + 1]), cc, mm), x0, x1);
-                f2_unpack(f2_fma(f2_pack(s[k0 + 2], s[k0 + 3]), cc, mm), x2, x3);
+                f2_unpack(f2_fma(f2_pack(s[k0], s[k0 + 1]), cc, mm8), x0, x1);
+                f2_unpack(f2_fma(f2_pack(s[k0 + 2], s[k0 + 3]), cc, mm8), x2, x3);
                 if (kEmu && emu_pair<C::EMU>(i)) {
                   f2_unpack(exp2_poly_x2(x0, x1), p0, p1);
                   f2_unpack(exp2_poly_x2(x2, x3), p2, p3);
@@ -581,14 +619,21 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                   p2 = ex2_approx(x2);
                   p3 = ex2_approx(x3);
                 }
-                const uint32_t lo = pack_e4m3x2(kP8Scale * p0, kP8Scale * p1);
-                const uint32_t hi = pack_e4m3x2(kP8Scale * p2, kP8Scale * p3);
+                // with the fold, p is already 256 p (and so are both sums)
+                constexpr float ps = ATTN_FWD_FP8FOLD ? 1.0f : kP8Scale;
+                const uint32_t lo = pack_e4m3x2(ps * p0, ps * p1);
+                const uint32_t hi = pack_e4m3x2(ps * p2, ps * p3);
                 pk[i] = lo | (hi << 16);
-                float q0, q1, q2, q3;
-                unpack_e4m3x2(lo, q0, q1);
-                unpack_e4m3x2(hi, q2, q3);
                 sf[i & 3] = f2_add(sf[i & 3], f2_add(f2_pack(p0, p1), f2_pack(p2, p3)));
-                sb[i & 3] = f2_add(sb[i & 3], f2_add(f2_pack(q0, q1), f2_pack(q2, q3)));
+                if constexpr (ATTN_FWD_MIXADD) {
+                  add_f16x2_f32(e4m3x2_to_f16x2(lo), sbf[0], sbf[1]);
+                  add_f16x2_f32(e4m3x2_to_f16x2(hi), sbf[2], sbf[3]);
+                } else {
+                  float q0, q1, q2, q3;
+                  unpack_e4m3x2(lo, q0, q1);
+                  unpack_e4m3x2(hi, q2, q3);
+                  sb[i & 3] = f2_add(sb[i & 3], f2_add(f2_pack(q0, q1), f2_pack(q2, q3)));
+                }
               }
               tmem_st16(tS + ch * 16, pk);
               publish(ch);
@@ -602,7 +647,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           f2_unpack(f2_add(f2_add(sf[0], sf[1]), f2_add(sf[2], sf[3])), a0, a1);
           f2_unpack(f2_add(f2_add(sb[0], sb[1]), f2_add(sb[2], sb[3])), b0, b1);
           l_run += a0 + a1;
-          lb_run += b0 + b1;
+          lb_run += (b0 + b1) + ((sbf[0] + sbf[1]) + (sbf[2] + sbf[3]));
         }
       }
       if (ok) {
@@ -640,7 +685,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
           }
           if (valid) {
-            const float lse = (m_run + __log2f(l_run)) * 0.69314718055994530942f;
+            // with the e4m3 fold, l_run sums 256 p
+            constexpr float kLFold = (FP8 && ATTN_FWD_FP8FOLD) ? 8.0f : 0.0f;
+            const float lse = (m_run + __log2f(l_run) - kLFold) * 0.69314718055994530942f;
             const size_t li = p.sv.cu ? size_t(it.h) * p.T + it.start + rpos
                                       : (size_t(it.seq) * p.Hq + it.h) * p.sv.S + rpos;
             p.lse[li] = lse;
