@@ -54,6 +54,13 @@ constexpr int kSlab = 128 * 128;
 #define ATTN_BWD_DSCHUNK 1
 #endif
 constexpr int kDsChunks = ATTN_BWD_DSCHUNK ? 4 : 1;
+// At D = 128 (dQ in the dP^T columns), dQ is issued as soon as the last dS chunk lands,
+// before that chunk's dK steps (1), so the dQ drain -- which the next tile's dP^T waits
+// for -- starts earlier; or after all of dK (0).  At D = 64 dQ has columns of its own and
+// always comes after dK.
+#ifndef ATTN_BWD_DQFIRST
+#define ATTN_BWD_DQFIRST 1
+#endif
 
 struct Params {
   SeqView sv;
@@ -379,19 +386,24 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // dK += dS^T Q (dS^T K-major in shared memory), chunk by chunk as dS arrives:
         // chunk c covers query K steps 2c, 2c + 1 (warpgroup c / 2, local half c % 2).  The
         // two warpgroups run side by side, so their first halves are taken first.
-        for (int j = 0; j < kDsChunks && ok; ++j) {
-          const int c = kDsChunks == 4 ? ((j & 1) << 1) | (j >> 1) : 0;
-          if (!(ok = mbar_wait(&ds_full[c], it & 1, wc, kSiteDsFull))) break;
-          tc_fence_after();
+        auto chunk_of = [](int j) { return kDsChunks == 4 ? ((j & 1) << 1) | (j >> 1) : 0; };
+        auto issue_dK = [&](int c) {
 #pragma unroll
           for (int k2 = 0; k2 < 8 / kDsChunks; ++k2) {
             const int kk = c * (8 / kDsChunks) + k2;
             mma_ss(tmem + C::COL_DK, sdesc_sw128(dsb + (kk >> 2) * kSlab + (kk & 3) * 32, 16, 1024),
                    sdesc_sw128(qb + kk * 2048, kSlab, 1024), idKV, (it > 0 || kk > 0) ? 1u : 0u);
           }
+        };
+        constexpr bool kDqFirst = ATTN_BWD_DQFIRST && C::DQ_ALIAS;
+        constexpr int kEarly = kDqFirst ? kDsChunks - 1 : kDsChunks;  // dK chunks before dQ
+        for (int j = 0; j < kDsChunks && ok; ++j) {
+          if (!(ok = mbar_wait(&ds_full[chunk_of(j)], it & 1, wc, kSiteDsFull))) break;
+          tc_fence_after();
+          if (j < kEarly) issue_dK(chunk_of(j));
         }
         if (!ok) break;
-        mma_commit(&q_empty[st]);
+        if (!kDqFirst) mma_commit(&q_empty[st]);
         if (!C::DQ_ALIAS && it > 0 && !(ok = mbar_wait(dq_free, (it - 1) & 1, wc, kSiteDqFree))) break;
         tc_fence_after();
 #pragma unroll
@@ -399,6 +411,12 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           mma_ss(tmem + C::COL_DQ, sdesc_sw128(dsb + kk * 2048, 16384, 1024),
                  sdesc_sw128(kb + kk * 2048, kSlab, 1024), idQ, kk > 0 ? 1u : 0u);
         mma_commit(dq_full);
+        if (kDqFirst) {
+          // the last chunk's dK steps; q_empty then also tells the P/dS warps that every
+          // read of this tile's dS buffer has been issued and completed
+          issue_dK(chunk_of(kDsChunks - 1));
+          mma_commit(&q_empty[st]);
+        }
       }
       if (ok) mma_commit(dkv_final);
       mma_commit(drain);
@@ -484,8 +502,13 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       // dS^T = P^T * (dP^T - Delta), written as bf16 into shared memory once the previous
       // dQ MMA has finished reading that buffer.  The one buffer is the A operand of both
       // MMAs that use dS: MN-major dS for dQ = dS K, K-major dS^T for dK += dS^T Q.
-      ok = __all_sync(0xffffffffu, mbar_wait(dp_full, it & 1, wc, kSiteDpFull) &&
-                                       (it == 0 || mbar_wait(dq_full, (it - 1) & 1, wc, kSiteDqFull)));
+      // The dS buffer is free once the previous tile's dQ (and, with dQ first, its last dK
+      // steps: q_empty of that tile) have read it.
+      ok = __all_sync(0xffffffffu,
+                      mbar_wait(dp_full, it & 1, wc, kSiteDpFull) &&
+                      (it == 0 || mbar_wait(dq_full, (it - 1) & 1, wc, kSiteDqFull)) &&
+                      (!(ATTN_BWD_DQFIRST && C::DQ_ALIAS) || it == 0 ||
+                       mbar_wait(&q_empty[(it - 1) & 1], ((it - 1) >> 1) & 1, wc, kSiteQEmpty)));
       if (!ok) break;
       tc_fence_after();
       // dP^T in two halves: the second loads while the first half's dS^T is computed.
