@@ -67,3 +67,34 @@ def test_clock_summary_keeps_the_timed_window_only():
     c = bench.summarize_clocks(lines, t0, t1)
     assert c["samples"] == 2 and c["window"].startswith("nearest")
     assert bench.summarize_clocks(["nothing parseable\n"], t0, t1)["samples"] == 0
+
+
+def test_traffic_record_follows_its_kernel_sources(tmp_path, monkeypatch):
+    """A DRAM-traffic record is reported only while the sources its kernel is built from
+    hash to the record's sha1; a change to another kernel's source leaves it valid."""
+    import shutil
+    import bench
+
+    csrc = os.path.join(ROOT, "long_context_attention_fwd_b200", "csrc")
+    root = tmp_path / "repo"
+    (root / "long_context_attention_fwd_b200").mkdir(parents=True)
+    shutil.copytree(csrc, root / "long_context_attention_fwd_b200" / "csrc")
+    (root / "profiles").mkdir()
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    wl = "some_workload"
+    rec = {"workloads": {wl: {k: {"dram_bytes_per_launch": 1000 + i, "sources_sha1": bench.kernel_sources_sha1(k)}
+                              for i, k in enumerate(bench.KERNEL_SOURCES)}}}
+    (root / "profiles" / "traffic.json").write_text(json.dumps(rec))
+    assert bench.measured_traffic(wl, "attn_bwd_kernel") == 1001
+    assert bench.measured_traffic(wl, "attn_fwd_kernel") == 1000
+    assert bench.measured_traffic("other_workload", "attn_bwd_kernel") is None
+    # edit the forward's own header: its record goes stale, the backward's stays
+    fwd = root / "long_context_attention_fwd_b200" / "csrc" / "attn_fwd.cuh"
+    fwd.write_text(fwd.read_text() + "\n// edited\n")
+    assert bench.measured_traffic(wl, "attn_fwd_kernel") is None
+    assert bench.measured_traffic(wl, "attn_bwd_kernel") == 1001
+    # a shared header invalidates both
+    ptx = root / "long_context_attention_fwd_b200" / "csrc" / "sm100_ptx.cuh"
+    ptx.write_text(ptx.read_text() + "\n// edited\n")
+    assert bench.measured_traffic(wl, "attn_bwd_kernel") is None
+
