@@ -739,9 +739,10 @@ def run_gpu(args, w: I.Workload):
 def run_profile_case(args):
     """One launch of the forward and/or backward on a reduced synthetic problem, for ncu
     captures that must stay small (a few GB on the device, one launch of each kernel):
-    --profile B,Hq,Hkv,S,D [--profile-op fwd|fwd8|bwd|both|decode] [--profile-outliers]
-    (fwd8: two e4m3 forward launches after one bf16 one; decode: B sequences of S cached
-    keys, two decode steps).  Inputs are
+    --profile B,Hq,Hkv,S,D [--profile-op fwd|fwd8|bwd|both|decode|merge|relayout]
+    [--profile-outliers] (fwd8: two e4m3 forward launches after one bf16 one; decode: B
+    sequences of S cached keys, two decode steps; merge: two merges of 4 partials shaped
+    like the forward's output; relayout: q into 4 head groups, twice).  Inputs are
     drawn on the GPU (N(0,1) * 0.5, or N(0,1) with 1% of q, k entries x8); the backward
     needs the forward's output, so --profile-op bwd also launches the forward once."""
     import torch
@@ -762,6 +763,23 @@ def run_profile_case(args):
         if st != capi.ATTN_OK:
             raise RuntimeError(f"device status {capi.strerror(st)} site={site:#x}")
         print(json.dumps({"profile_case": [B, Hq, Hkv, S, D], "op": "decode", "status": "ok"}))
+        return 0
+    if args.profile_op in ("merge", "relayout"):
+        g = torch.Generator(device=dev).manual_seed(20261203)
+        x = (torch.randn((B, S, Hq, D), generator=g, device=dev) * 0.5).bfloat16()
+        parts = [x.clone() for _ in range(4)] if args.profile_op == "merge" else None
+        lse = torch.randn((B, Hq, S), generator=g, device=dev)
+        lses = [lse + 0.25 * j for j in range(4)]
+        for _ in range(2):
+            if args.profile_op == "merge":
+                ops.attn_merge(parts, lses)
+            else:
+                ops.transpose_blocks(x, B * S, 4)
+        torch.cuda.synchronize()
+        st, site = capi.attn_device_status(None)
+        if st != capi.ATTN_OK:
+            raise RuntimeError(f"device status {capi.strerror(st)} site={site:#x}")
+        print(json.dumps({"profile_case": [B, Hq, Hkv, S, D], "op": args.profile_op, "status": "ok"}))
         return 0
     g = torch.Generator(device=dev).manual_seed(20261203)
     mult = 1.0 if args.profile_outliers else 0.5
@@ -801,7 +819,8 @@ def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--profile", default=None, metavar="B,Hq,Hkv,S,D",
                     help="one launch on a reduced synthetic problem, for ncu captures")
-    ap.add_argument("--profile-op", default="both", choices=["fwd", "fwd8", "bwd", "both", "decode"])
+    ap.add_argument("--profile-op", default="both",
+                    choices=["fwd", "fwd8", "bwd", "both", "decode", "merge", "relayout"])
     ap.add_argument("--profile-outliers", action="store_true")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
